@@ -1,0 +1,250 @@
+"""Pins of the oracle's attention: invariants, identities, special cases, bounds.
+
+- smooth_k invariant: subtracting the per-channel K mean shifts every logit of
+  a row by the same constant, so fp64 softmax attention is unchanged
+  ("sageattention" package page, Quickstart: smooth_k=True by default).
+- Q smoothing: Q'K'^T + 1 dS^T restores Q K'^T exactly ("SageAttention2:
+  Technical report", section 2: subtract the channel mean of Q and V).
+- V smoothing: P(V - 1 mu^T) + 1 mu^T = P V for row-stochastic P (same section).
+- Special cases with a closed form: Q = 0 gives the mean of the (dequantised)
+  visible V rows (prefix means when causal); Nkv = 1 gives that row; constant
+  V gives the constant up to the FP8 rounding of P.
+- The fp64 exact attention equals PyTorch's scaled_dot_product_attention in
+  fp64 (library routine), including causal masking and GQA.
+- The quantised mirror stays within the error the FP8/INT8 steps allow of the
+  exact result (relative L1 <= 0.06, cosine >= 0.998 on iid data: FP8 e4m3 has
+  a relative step of 2^-3, i.e. ~3.6% rms rounding error per operand; see the
+  measured values in the design notes), also when block scales differ by
+  orders of magnitude and when the running max grows tile after tile.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_attention_subtract_b200.workloads import generate, random_problem
+
+
+def _problem(w, **kw):
+    d = dict(B=w.B, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, Nkv=w.Nkv, D=w.D, layout=w.layout, dtype=w.dtype,
+             is_causal=w.is_causal, smooth_k=w.smooth_k, smooth_q=w.smooth_q, smooth_v=w.smooth_v)
+    d.update(kw)
+    return oracle.Problem(**d)
+
+
+def _hnd(pr, x):
+    x = oracle.to_double(pr, x)
+    return x if pr.layout == "HND" else x.transpose(0, 2, 1, 3)
+
+
+def _tiled(pr, full_hnd):
+    """[B,H,N,D] -> [n_tiles,128,D] in all_tiles order."""
+    t = oracle.all_tiles(pr)
+    out = np.zeros((len(t), 128, pr.D))
+    for n, (b, h, qt) in enumerate(t):
+        i0, i1 = qt * 128, min(qt * 128 + 128, pr.Nq)
+        out[n, : i1 - i0] = full_hnd[b, h, i0:i1]
+    return out
+
+
+def _softmax_attn(Q, K, V, scale, causal, group):
+    K = np.repeat(K, group, axis=1)
+    V = np.repeat(V, group, axis=1)
+    s = np.einsum("bhid,bhjd->bhij", Q, K) * scale
+    if causal:
+        i = np.arange(Q.shape[2])[:, None]
+        j = np.arange(K.shape[2])[None, :]
+        s = np.where(j <= i, s, -np.inf)
+    s = s - s.max(-1, keepdims=True)
+    p = np.exp(s)
+    return np.einsum("bhij,bhjd->bhid", p / p.sum(-1, keepdims=True), V)
+
+
+def _rel_l1(a, b):
+    return np.abs(a - b).sum() / np.abs(b).sum()
+
+
+def _cos(a, b):
+    return (a * b).sum() / np.linalg.norm(a) / np.linalg.norm(b)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_exact_attention_matches_torch_sdpa_fp64(causal):
+    w = random_problem(2, 4, 2, 200, 200 if causal else 333, 64, dtype="fp16", seed=4)
+    pr = _problem(w, is_causal=causal)
+    q, k, v = generate(w)
+    Q, K, V = (torch.from_numpy(_hnd(pr, x)) for x in (q, k, v))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        Q, K, V, is_causal=causal, scale=float(pr.resolved_sm_scale()), enable_gqa=True).numpy()
+    got = oracle.exact_attention_tiles(pr, q, k, v, oracle.all_tiles(pr))
+    assert np.max(np.abs(got - _tiled(pr, ref))) < 1e-12
+
+
+def test_smooth_k_invariant_fp64():
+    w = random_problem(1, 2, 2, 256, 256, 64, dtype="fp16", seed=0, k_offset_sigma=3.0)
+    pr = _problem(w)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v)
+    Q, K, V = _hnd(pr, q), _hnd(pr, k), _hnd(pr, v)
+    s = float(pr.resolved_sm_scale())
+    a = _softmax_attn(Q, K, V, s, False, 1)
+    b = _softmax_attn(Q, K - pre["mean_k"][:, :, None, :], V, s, False, 1)
+    assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(a))
+    # subtracting a per-*token* quantity instead would not be invariant
+    c = _softmax_attn(Q, K - K.mean(axis=3, keepdims=True), V, s, False, 1)
+    assert np.max(np.abs(a - c)) > 1e-3
+
+
+def test_q_smoothing_correction_restores_qk():
+    w = random_problem(1, 4, 2, 300, 200, 96, dtype="bf16", seed=6, k_offset_sigma=3.0)
+    pr = _problem(w, smooth_q=True)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v)
+    Q = _hnd(pr, q)
+    for b, h, qt in [(0, 0, 0), (0, 3, 2), (0, 1, 1)]:
+        kp = pre["kp"][0, h // 2].astype(np.float64)
+        i0, i1 = qt * 128, min(qt * 128 + 128, pr.Nq)
+        Qb = Q[b, h, i0:i1]
+        mq = pre["mq"][b, h, qt].astype(np.float64)
+        dS = oracle.delta_s(pr, pre, b, h, qt)
+        lhs = (Qb - mq) @ kp.T + dS[None, :]
+        rhs = Qb @ kp.T
+        assert np.max(np.abs(lhs - rhs)) <= 1e-12 * np.max(np.abs(rhs))
+        # dropping the correction is far off
+        assert np.max(np.abs((Qb - mq) @ kp.T - rhs)) > 1e-3
+
+
+def test_v_smoothing_identity():
+    w = random_problem(1, 2, 2, 128, 200, 64, dtype="fp16", seed=7)
+    pr = _problem(w, smooth_v=True)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v)
+    V = _hnd(pr, v)[0, 0]
+    mu = pre["mean_v"][0, 0].astype(np.float64)
+    rng = np.random.default_rng(0)
+    P = rng.random((128, 200))
+    P /= P.sum(1, keepdims=True)
+    assert np.max(np.abs(P @ (V - mu) + mu - P @ V)) < 1e-12
+
+
+@pytest.mark.parametrize("causal,layout,Nq,Nkv,Hq,Hkv,D", [
+    (False, "HND", 256, 200, 4, 2, 64),
+    (True, "HND", 300, 300, 4, 1, 128),
+    (True, "NHD", 260, 260, 2, 2, 96),
+    (False, "NHD", 130, 700, 6, 3, 64),
+])
+def test_zero_q_gives_mean_of_visible_v(causal, layout, Nq, Nkv, Hq, Hkv, D):
+    w = random_problem(2, Hq, Hkv, Nq, Nkv, D, layout=layout, dtype="bf16", seed=8)
+    pr = _problem(w, is_causal=causal, smooth_v=True)
+    q, k, v = generate(w)
+    q = np.zeros_like(q)
+    pre = oracle.prepass(pr, q, k, v)
+    table = oracle.e4m3_decode_table()
+    Vd = table[pre["v8"]] * pre["v_scale"][:, :, None, :] + pre["mean_v"][:, :, None, :]
+    Vd = np.repeat(Vd, Hq // Hkv, axis=1)
+    if causal:
+        want = np.cumsum(Vd, axis=2)[:, :, :Nq] / np.arange(1, Nq + 1)[None, None, :, None]
+    else:
+        want = np.broadcast_to(Vd.mean(axis=2, keepdims=True), (2, Hq, Nq, D))
+    got = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))
+    assert np.max(np.abs(got - _tiled(pr, want))) <= 1e-6 * np.max(np.abs(want))
+
+
+def test_single_key_gives_that_row():
+    w = random_problem(1, 2, 1, 200, 1, 128, dtype="fp16", seed=9)
+    pr = _problem(w)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v)
+    table = oracle.e4m3_decode_table()
+    row = table[pre["v8"][0, 0, 0]] * pre["v_scale"][0, 0]
+    got = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))
+    valid = np.concatenate([got[0], got[1, :72], got[2], got[3, :72]])
+    assert np.max(np.abs(valid - row)) <= 1e-6 * np.max(np.abs(row))
+
+
+def test_constant_v_gives_the_constant():
+    w = random_problem(1, 2, 2, 256, 500, 64, dtype="fp16", seed=10)
+    pr = _problem(w)
+    q, k, v = generate(w)
+    const = np.linspace(-3, 3, 64).astype(np.float16)
+    v = np.broadcast_to(const.view(np.uint16), v.shape).copy()
+    pre = oracle.prepass(pr, q, k, v)
+    got = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))
+    c = const.astype(np.float64)
+    # sum of FP8-rounded p over sum of p is within the e4m3 relative step 2^-4 of 1
+    assert np.all(np.abs(got - c) <= 2.0 ** -4 * np.abs(c) + 1e-12)
+
+
+CASES = [
+    dict(args=(1, 2, 2, 256, 256, 64), dtype="fp16"),
+    dict(args=(2, 4, 2, 300, 200, 96), dtype="bf16"),
+    dict(args=(1, 4, 1, 384, 384, 128), dtype="bf16", is_causal=True),
+    dict(args=(1, 2, 2, 256, 512, 64), dtype="fp16", smooth_k=False),
+    dict(args=(1, 2, 2, 256, 512, 64), dtype="fp16", smooth_q=True, smooth_v=True),
+    dict(args=(1, 2, 2, 200, 390, 64), dtype="bf16", layout="NHD", is_causal=True),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[str(i) for i in range(len(CASES))])
+def test_mirror_within_quantisation_error_of_exact(case):
+    flags = {k: v for k, v in case.items() if k in ("is_causal", "smooth_k", "smooth_q", "smooth_v")}
+    w = random_problem(*case["args"], layout=case.get("layout", "HND"), dtype=case["dtype"], seed=3,
+                       k_offset_sigma=3.0)
+    pr = _problem(w, **flags)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v)
+    t = oracle.all_tiles(pr)
+    m = oracle.attention_tiles(pr, pre, t)
+    e = oracle.exact_attention_tiles(pr, q, k, v, t)
+    assert _rel_l1(m, e) <= 0.06 and _cos(m, e) >= 0.998
+
+
+def test_mirror_uses_the_right_block_scales():
+    # K blocks (64 tokens) and Q blocks (128 tokens) with magnitudes that
+    # differ by orders of magnitude: a wrong block index in the scale lookup
+    # changes logits by large factors.
+    w = random_problem(1, 2, 2, 384, 384, 64, dtype="fp16", seed=12, k_offset_sigma=0.0)
+    pr = _problem(w, smooth_k=False)
+    q, k, v = generate(w)
+    Q, K = oracle.to_double(pr, q), oracle.to_double(pr, k)
+    kscale = np.array([0.02, 1.0, 0.1, 3.0, 0.5, 0.05])
+    qscale = np.array([0.1, 2.0, 0.5])
+    K = K * np.repeat(kscale, 64)[None, None, :, None]
+    Q = Q * np.repeat(qscale, 128)[None, None, :, None]
+    q = Q.astype(np.float16).view(np.uint16)
+    k = K.astype(np.float16).view(np.uint16)
+    pre = oracle.prepass(pr, q, k, v)
+    t = oracle.all_tiles(pr)
+    m = oracle.attention_tiles(pr, pre, t)
+    e = oracle.exact_attention_tiles(pr, q, k, v, t)
+    assert _rel_l1(m, e) <= 0.06 and _cos(m, e) >= 0.998
+
+
+def test_mirror_rescales_when_max_grows():
+    # Logits rise tile after tile, so the running max grows in every KV tile
+    # and the O / l rescaling is exercised on every step.
+    w = random_problem(1, 1, 1, 128, 1024, 64, dtype="fp16", seed=13, k_offset_sigma=0.0)
+    pr = _problem(w, smooth_k=False)
+    q, k, v = generate(w)
+    rng = np.random.default_rng(1)
+    u = rng.standard_normal(64)
+    u /= np.linalg.norm(u)
+    Q = 0.3 * rng.standard_normal((1, 1, 128, 64)) + 2.0 * u
+    ramp = np.linspace(0, 6.0, 1024)[:, None]
+    K = 0.3 * rng.standard_normal((1, 1, 1024, 64)) + ramp * u
+    q = Q.astype(np.float16).view(np.uint16)
+    k = K.astype(np.float16).view(np.uint16)
+    pre = oracle.prepass(pr, q, k, v)
+    t = oracle.all_tiles(pr)
+    m = oracle.attention_tiles(pr, pre, t)
+    e = oracle.exact_attention_tiles(pr, q, k, v, t)
+    assert _rel_l1(m, e) <= 0.06 and _cos(m, e) >= 0.998
+
+
+def test_mirror_is_layout_invariant():
+    w = random_problem(2, 4, 2, 200, 300, 64, dtype="bf16", seed=14)
+    pr_h, pr_n = _problem(w, is_causal=False), _problem(w.with_(layout="NHD"))
+    a = oracle.attention_tiles(pr_h, oracle.prepass(pr_h, *generate(w)), oracle.all_tiles(pr_h))
+    b = oracle.attention_tiles(pr_n, oracle.prepass(pr_n, *generate(w.with_(layout="NHD"))),
+                               oracle.all_tiles(pr_n))
+    assert np.array_equal(a, b)
