@@ -1,0 +1,317 @@
+"""Benchmark of the quantized attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one whole pass (smoothing + quantisation pre-pass, then the
+attention kernel) over one batch of the named synthetic workload (default:
+B4 H32 N4096 D128 bf16 HND, non-causal), inputs resident in HBM.  The metric
+is attention TOPS = 4*B*Hq*Nq*Nkv*D / time (halved for causal), whole job.
+Under torchrun (N > 1) every rank runs the same workload on its own GPU
+(independent replicas, no collective in the data path: the pass does not
+shard across GPUs); the time is the max over ranks.
+
+Reported beside the value: the attention kernel's roofline (tensor-bound,
+8-bit peak derived from the measured bf16 GEMM peak x 2, the nominal 8-bit /
+16-bit ratio), the end-to-end number through the public API with host
+buffers, SM clocks sampled during the timed region, and the CPU oracle timed
+on a bounded sample (``cpu_baseline``).  ``--impl reference`` times the CPU
+oracle itself on the same workload, one bounded sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from quantized_attention_subtract_b200.workloads import WORKLOADS, Workload, generate  # noqa: E402
+
+METRIC = "attention TOPS (4*B*H*Nq*Nkv*d/s) at N=4K-32K, d=128; % of B200 tensor peak"
+DEFAULT_WORKLOAD = "mha_n4096_d128_bf16"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return float(m["bf16_tflops"]), float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 1590.0, 6650.0, "fallback"
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _oracle_problem(w: Workload):
+    import oracle
+    return oracle.Problem(B=w.B, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, Nkv=w.Nkv, D=w.D, layout=w.layout,
+                          dtype=w.dtype, is_causal=w.is_causal, smooth_k=w.smooth_k,
+                          smooth_q=w.smooth_q, smooth_v=w.smooth_v)
+
+
+def oracle_sample(w: Workload, kv_heads: int):
+    """Time the CPU oracle (pre-pass + tiled attention) on the first `kv_heads`
+    kv heads of batch 0 with all their query heads and tiles.  Returns
+    (tops, seconds, description, threads)."""
+    import oracle
+    group = w.Hq // w.Hkv
+    sub = w.with_(B=1, Hkv=kv_heads, Hq=kv_heads * group)
+    q, k, v = generate(sub)
+    pr = _oracle_problem(sub)
+    t0 = time.perf_counter()
+    pre = oracle.prepass(pr, q, k, v)
+    oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))
+    dt = time.perf_counter() - t0
+    desc = (f"batch 0, kv heads 0..{kv_heads - 1} ({sub.Hq} query heads, all {pr.nqb} query tiles "
+            f"each) of {w.name}: pre-pass + tiled quantised attention")
+    return sub.ops / dt / 1e12, dt, desc, oracle.num_threads()
+
+
+def _sample_heads(w: Workload, target_s: float) -> int:
+    """kv heads of batch 0 whose oracle run takes about target_s seconds."""
+    import oracle
+    per_head = None
+    try:
+        _, dt, _, _ = oracle_sample(w.with_(Nq=min(w.Nq, 256)), 1)
+        per_head = dt * (w.Nq / min(w.Nq, 256))
+    except Exception:
+        per_head = 1.0
+    n = max(1, int(target_s / max(per_head, 1e-3)))
+    return min(n, w.Hkv)
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_reference(args, w: Workload):
+    """The CPU oracle timed as the reference arm (rank 0 only)."""
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    heads = _sample_heads(w, 2.0)
+    for _ in range(args.warmup):
+        oracle_sample(w, heads)
+    times, tops = [], []
+    desc, threads = "", 1
+    for _ in range(args.steps):
+        t, dt, desc, threads = oracle_sample(w, heads)
+        times.append(dt)
+        tops.append(t)
+    value = float(np.mean(tops))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * float(np.mean(times)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "i8xi8->i64 (QK), e4m3xe4m3->f64 (PV)", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nkv": w.Nkv,
+                   "D": w.D, "layout": w.layout, "causal": w.is_causal, "smooth_k": w.smooth_k},
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, w: Workload):
+    import torch
+    from quantized_attention_subtract_b200 import binding, sageattn
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    q, k, v = generate(w)
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).to(dev).view(
+        torch.float16 if w.dtype == "fp16" else torch.bfloat16)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    out = torch.empty_like(qd)
+    p = binding.make_params(qd, kd, vd, out, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q,
+                            w.smooth_v)
+    ws = binding.alloc_workspace(p, dev)
+    stream = torch.cuda.current_stream(dev)
+    in_bytes = qd.numel() * 2 + kd.numel() * 2 + vd.numel() * 2
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- warm-up, then K timed steps of the whole pass
+    for _ in range(args.warmup):
+        binding.attn_fwd(p, dev)
+    barrier()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            binding.attn_fwd(p, dev)
+        end.record(stream)
+        barrier()
+        step_ms = start.elapsed_time(end) / args.steps
+        # ---- the attention kernel alone (dominant kernel), per-launch events
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            a.record(stream)
+            binding.attn_quantized(p, dev)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        # ---- the pre-pass alone
+        for a, b in evs:
+            a.record(stream)
+            binding.quantize(p, dev)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        pre_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    clocks = clk.summary()
+    assert binding.device_status(p) == 0, "device status nonzero"
+
+    # max over ranks
+    t = torch.tensor([step_ms, attn_ms, pre_ms], device=dev)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    step_ms, attn_ms, pre_ms = (float(x) for x in t.tolist())
+
+    # ---- end to end through the public API with pinned host buffers
+    qh, kh, vh = (x.cpu().pin_memory() for x in (qd, kd, vd))
+    oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    for _ in range(2):
+        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh)
+    e1.record(stream)
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
+    if pg is not None:
+        pg.all_reduce(e2e_ms, op=pg.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    bf16_tflops, hbm_gbs, peak_src = _peaks()
+    peak8 = 2.0 * bf16_tflops  # 8-bit dense = 2 x bf16 dense (nominal 4.5 / 2.25 PFLOP/s)
+    achieved = w.ops / (attn_ms * 1e-3) / 1e12
+    value = world * w.ops / (step_ms * 1e-3) / 1e12
+    kernels_per_step = 3 + (1 if w.smooth_q else 0)  # kv_stats, quantize, (delta_s), attention
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nkv": w.Nkv,
+                   "D": w.D, "layout": w.layout, "input_dtype": w.dtype, "causal": w.is_causal,
+                   "smooth_k": w.smooth_k, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs {in_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
+                     "peak": peak8, "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 x 2 (burst)", "attn_ms": attn_ms,
+                     "prepass_ms": pre_ms,
+                     "prepass_gbs": 3 * (qd.numel() + kd.numel() + vd.numel()) / (pre_ms * 1e-3) / 1e9},
+        "e2e": {"value": world * w.ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * 2},
+        "clocks": clocks,
+        "gpu_launches": kernels_per_step * args.steps,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        heads = _sample_heads(w, 12.0)
+        tops, dt, desc, threads = oracle_sample(w, heads)
+        line["cpu_baseline"] = {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                                "sample": desc + f" ({dt:.1f} s)"}
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

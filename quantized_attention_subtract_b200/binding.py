@@ -1,0 +1,276 @@
+"""Thin ctypes binding of libsage_b200.so (the C ABI in include/sage_b200.h).
+
+Argument marshalling only: every step of the pass runs in the library's CUDA
+kernels.  PyTorch supplies device memory (inputs, output, workspace) and the
+current stream.  There is no fallback: if the library is missing or the
+device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsage_b200.so")
+
+SAGE_OK = 0
+STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
+                3: "SAGE_ERR_ALIGNMENT", 4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_DEVICE_TIMEOUT",
+                6: "SAGE_ERR_WORKSPACE"}
+
+# Every symbol include/sage_b200.h declares.
+EXPORTED = ["sage_abi_version", "sage_status_string", "sage_workspace_size", "sage_workspace_view",
+            "sage_attn_fwd", "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
+            "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop", "sage_debug_wait_timeout",
+            "sage_get_device_status"]
+
+
+class SageError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+class Params(ctypes.Structure):
+    """Mirror of sage_attn_params_t."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("out", ctypes.c_void_p),
+        ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+        ("Nq", ctypes.c_int32), ("Nkv", ctypes.c_int32), ("D", ctypes.c_int32),
+        ("q_strides", ctypes.c_int64 * 4), ("k_strides", ctypes.c_int64 * 4),
+        ("v_strides", ctypes.c_int64 * 4), ("o_strides", ctypes.c_int64 * 4),
+        ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("is_causal", ctypes.c_int32), ("smooth_k", ctypes.c_int32),
+        ("smooth_q", ctypes.c_int32), ("smooth_v", ctypes.c_int32),
+        ("sm_scale", ctypes.c_float),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+class WorkspaceView(ctypes.Structure):
+    """Mirror of sage_workspace_view_t."""
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("q8", "k8", "v8t", "q_scale", "k_scale", "v_scale", "mean_k", "mean_v", "mq",
+                 "dsk", "status")] + [("Dp", ctypes.c_int32), ("Nq_pad", ctypes.c_int32),
+                                      ("Nkv_pad", ctypes.c_int32)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib():
+    """Load libsage_b200.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"CUDA library missing: {LIB_PATH} (run "
+                                   "`python -m quantized_attention_subtract_b200.build`)")
+            L = ctypes.CDLL(LIB_PATH)
+            P = ctypes.POINTER(Params)
+            vp, i32 = ctypes.c_void_p, ctypes.c_int32
+            L.sage_abi_version.restype = i32
+            L.sage_status_string.restype = ctypes.c_char_p
+            L.sage_status_string.argtypes = [ctypes.c_int]
+            L.sage_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
+            L.sage_workspace_view.argtypes = [P, ctypes.POINTER(WorkspaceView)]
+            for f in (L.sage_attn_fwd, L.sage_quantize, L.sage_attn_quantized):
+                f.argtypes = [P, vp]
+            L.sage_debug_dump_s.argtypes = [P, i32, i32, i32, i32, vp, vp]
+            L.sage_debug_pv.argtypes = [P, i32, i32, i32, vp, vp, vp]
+            L.sage_debug_e4m3.argtypes = [vp, vp, ctypes.c_int64, vp]
+            L.sage_debug_mma_loop.argtypes = [i32, i32, vp, vp]
+            L.sage_get_device_status.argtypes = [P, ctypes.POINTER(i32)]
+            L.sage_debug_wait_timeout.argtypes = [vp, vp]
+            for name in ("sage_workspace_size", "sage_workspace_view", "sage_attn_fwd",
+                         "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
+                         "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop",
+                         "sage_debug_wait_timeout", "sage_get_device_status"):
+                getattr(L, name).restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != SAGE_OK:
+        raise SageError(code, what)
+
+
+def _stream(device: torch.device | None = None) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dims(x: torch.Tensor, layout: str):
+    if x.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    if layout == "HND":
+        B, H, N, D = x.shape
+    elif layout == "NHD":
+        B, N, H, D = x.shape
+    else:
+        raise ValueError(f"tensor_layout must be 'HND' or 'NHD', got {layout!r}")
+    return B, H, N, D
+
+
+def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scale=None,
+                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None) -> Params:
+    """Fill sage_attn_params_t from torch tensors (no copies, strides as given)."""
+    B, Hq, Nq, D = _dims(q, tensor_layout)
+    Bk, Hkv, Nkv, Dk = _dims(k, tensor_layout)
+    if v.shape != k.shape:
+        raise ValueError("k and v must have the same shape")
+    if (Bk, Dk) != (B, D):
+        raise ValueError("q and k disagree on batch or head_dim")
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype float16 or bfloat16")
+    p = Params()
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.out = out.data_ptr() if out is not None else None
+    p.B, p.Hq, p.Hkv, p.Nq, p.Nkv, p.D = B, Hq, Hkv, Nq, Nkv, D
+    for name, t in (("q_strides", q), ("k_strides", k), ("v_strides", v), ("o_strides", out)):
+        st = t.stride() if t is not None else (0, 0, 0, 1)
+        getattr(p, name)[:] = list(st)
+    p.layout = 0 if tensor_layout == "HND" else 1
+    p.dtype = 0 if q.dtype == torch.float16 else 1
+    p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
+                                                       int(bool(smooth_q)), int(bool(smooth_v)))
+    p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
+    if workspace is not None:
+        p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    return p
+
+
+def workspace_bytes(p: Params) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().sage_workspace_size(ctypes.byref(p), ctypes.byref(n)), "sage_workspace_size")
+    return int(n.value)
+
+
+def alloc_workspace(p: Params, device) -> torch.Tensor:
+    """A workspace of the right size (torch allocations are 512-byte aligned)."""
+    ws = torch.empty(workspace_bytes(p), dtype=torch.uint8, device=device)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    return ws
+
+
+def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
+             is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
+             smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Quantized attention forward: INT8 Q K^T, FP8 P V, on the current CUDA stream.
+
+    q: [B, Hq, Nq, D] ("HND") or [B, Nq, Hq, D] ("NHD"); k, v: same with Hkv, Nkv.
+    Host (CPU) tensors are copied to the current device and the result back.
+    """
+    host = not q.is_cuda
+    if host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be on the same device")
+    dev_out = torch.empty_like(q) if (out is None or host) else out
+    p = make_params(q, k, v, dev_out, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
+                    smooth_v)
+    if workspace is None:
+        workspace = alloc_workspace(p, q.device)
+    else:
+        p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(q.device)), "sage_attn_fwd")
+    if host:
+        res = out if out is not None else torch.empty(dev_out.shape, dtype=dev_out.dtype,
+                                                      pin_memory=True)
+        res.copy_(dev_out, non_blocking=True)
+        return res
+    return dev_out
+
+
+def quantize(p: Params, device) -> None:
+    _check(lib().sage_quantize(ctypes.byref(p), _stream(device)), "sage_quantize")
+
+
+def attn_quantized(p: Params, device) -> None:
+    _check(lib().sage_attn_quantized(ctypes.byref(p), _stream(device)), "sage_attn_quantized")
+
+
+def attn_fwd(p: Params, device) -> None:
+    _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(device)), "sage_attn_fwd")
+
+
+def workspace_views(p: Params, workspace: torch.Tensor) -> dict:
+    """torch views of the quantised tensors inside the workspace."""
+    w = WorkspaceView()
+    _check(lib().sage_workspace_view(ctypes.byref(p), ctypes.byref(w)), "sage_workspace_view")
+    base = workspace.data_ptr()
+
+    def view(addr, n, dtype, shape):
+        off = addr - base
+        esize = torch.tensor([], dtype=dtype).element_size()
+        return workspace[off: off + n * esize].view(dtype).view(*shape)
+
+    B, Hq, Hkv, D = p.B, p.Hq, p.Hkv, p.D
+    nqb, nkb = w.Nq_pad // 128, w.Nkv_pad // 64
+    out = dict(
+        q8=view(w.q8, B * Hq * w.Nq_pad * w.Dp, torch.int8, (B, Hq, w.Nq_pad, w.Dp)),
+        k8=view(w.k8, B * Hkv * w.Nkv_pad * w.Dp, torch.int8, (B, Hkv, w.Nkv_pad, w.Dp)),
+        v8t=view(w.v8t, B * Hkv * D * w.Nkv_pad, torch.uint8, (B, Hkv, D, w.Nkv_pad)),
+        q_scale=view(w.q_scale, B * Hq * nqb, torch.float32, (B, Hq, nqb)),
+        k_scale=view(w.k_scale, B * Hkv * nkb, torch.float32, (B, Hkv, nkb)),
+        v_scale=view(w.v_scale, B * Hkv * D, torch.float32, (B, Hkv, D)),
+        mean_k=view(w.mean_k, B * Hkv * D, torch.float32, (B, Hkv, D)),
+        mean_v=view(w.mean_v, B * Hkv * D, torch.float32, (B, Hkv, D)),
+        status=view(w.status, 1, torch.int32, (1,)),
+        Dp=w.Dp, Nq_pad=w.Nq_pad, Nkv_pad=w.Nkv_pad,
+    )
+    if w.mq:
+        out["mq"] = view(w.mq, B * Hq * nqb * D, torch.float32, (B, Hq, nqb, D))
+        out["dsk"] = view(w.dsk, B * Hq * nqb * w.Nkv_pad, torch.float32, (B, Hq, nqb, w.Nkv_pad))
+    return out
+
+
+def debug_dump_s(p: Params, b: int, h: int, qtile: int, ktile: int, device) -> torch.Tensor:
+    s = torch.empty((128, 128), dtype=torch.int32, device=device)
+    _check(lib().sage_debug_dump_s(ctypes.byref(p), b, h, qtile, ktile, ctypes.c_void_p(s.data_ptr()),
+                                   _stream(device)), "sage_debug_dump_s")
+    return s
+
+
+def debug_pv(p: Params, b: int, hkv: int, ktile: int, p8: torch.Tensor, device) -> torch.Tensor:
+    assert p8.dtype == torch.uint8 and p8.shape == (128, 128) and p8.is_contiguous()
+    o = torch.empty((128, p.D), dtype=torch.float32, device=device)
+    _check(lib().sage_debug_pv(ctypes.byref(p), b, hkv, ktile, ctypes.c_void_p(p8.data_ptr()),
+                               ctypes.c_void_p(o.data_ptr()), _stream(device)), "sage_debug_pv")
+    return o
+
+
+def debug_e4m3(x: torch.Tensor) -> torch.Tensor:
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    _check(lib().sage_debug_e4m3(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                 x.numel(), _stream(x.device)), "sage_debug_e4m3")
+    return out
+
+
+def debug_mma_loop(ctas: int, iters: int, sink: torch.Tensor) -> None:
+    """sink: int32 device tensor with at least ctas + 1 entries (the last one is a status word)."""
+    assert sink.dtype == torch.int32 and sink.numel() >= ctas + 1
+    _check(lib().sage_debug_mma_loop(ctas, iters, ctypes.c_void_p(sink.data_ptr()),
+                                     _stream(sink.device)), "sage_debug_mma_loop")
+
+
+def debug_wait_timeout(status: torch.Tensor) -> None:
+    """Run a bounded wait that nothing completes; status[0] becomes SAGE_ERR_DEVICE_TIMEOUT."""
+    assert status.dtype == torch.int32 and status.is_cuda
+    _check(lib().sage_debug_wait_timeout(ctypes.c_void_p(status.data_ptr()), _stream(status.device)),
+           "sage_debug_wait_timeout")
+
+
+def device_status(p: Params) -> int:
+    code = ctypes.c_int32(0)
+    _check(lib().sage_get_device_status(ctypes.byref(p), ctypes.byref(code)),
+           "sage_get_device_status")
+    return int(code.value)

@@ -1,0 +1,667 @@
+// attn_fwd.cu -- the quantized attention kernel for sm_100a.
+//
+// Computes, per (batch, query head, 128-row query tile), the flash-style
+// pass the SageAttention pages describe (INT8 Q K^T, FP8 P V; closerAI
+// ComfyUI blog, part 2; "sageattention" package page, "What it is"):
+//   S = q8 k8^T                    exact int32, tensor cores (kind::i8)
+//   s = S * q_scale * k_scale * sm_scale * log2(e)   (+ dS for smoothed Q)
+//   online softmax in base 2 with running max m and sum l
+//   P8 = e4m3(448 * 2^(s - m))     FP8 probabilities
+//   O += P8 v8                     fp32 accumulation, tensor cores (kind::f8f6f4)
+//   out = O * v_scale / l (+ mean_v), rounded to bf16 / fp16
+//
+// One CTA (192 threads) owns one query tile; two CTAs share an SM, so the
+// tensor core alternates between them while each runs its softmax.
+//   warp 0      TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ... into a
+//               3-stage shared-memory ring (order = MMA consumption order)
+//   warp 1      allocates 256 TMEM columns; lane 0 issues the MMAs:
+//               S_{j+1} = Q K_{j+1}^T as soon as softmax has read S_j, then
+//               O += P_j V_j once P_j is in shared memory
+//   warps 2-5   softmax: one query row per thread (TMEM lane), reads S with
+//               tcgen05.ld, writes P_j (swizzled, double-buffered) to shared
+//               memory, rescales its O row in TMEM when the max grows, and
+//               runs the epilogue
+// TMEM: S at columns [0,128), O at [128, 128 + D).
+// Causal tiles past the diagonal are skipped; keys >= Nkv and (causal)
+// keys > query are masked; rows >= Nq are computed but not stored.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace sage {
+namespace {
+
+template <int D>
+struct Cfg {
+  static constexpr int Dp = D == 64 ? 64 : 128;       // INT8 row length in smem / workspace
+  static constexpr int kQKSteps = D / 32;             // K=32 bytes per 8-bit MMA
+  static constexpr int kStages = 3;
+  static constexpr int kQBytes = 128 * Dp;
+  static constexpr int kKBytes = 128 * Dp;
+  static constexpr int kVBytes = D * 128;
+  static constexpr int kStageBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
+  static constexpr int kPBytes = 128 * 128;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffRing = kOffQ + kQBytes;
+  static constexpr int kOffP = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffBar = kOffP + 2 * kPBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmem = kOffBar + kBarBytes + 1024;   // +1024: base alignment slack
+  static constexpr uint32_t kTmemCols = 256;
+  static constexpr int kThreads = 192;
+};
+
+// Barrier slots (8 bytes each) inside the barrier area.
+enum Bar {
+  kBarQ = 0,
+  kBarFull = 1,    // + stage (3)
+  kBarEmpty = 4,   // + stage (3)
+  kBarSFull = 7,
+  kBarSEmpty = 8,
+  kBarPFull = 9,   // + buffer (2)
+  kBarPVDone = 11, // + buffer (2)
+  kBarFinal = 13,
+  kNumBars = 14
+};
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int *status) {
+  const bool ok = mbar_wait(bar, parity, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+  return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+template <int D, bool kSmoothQ>
+__global__ void __launch_bounds__(192, 2)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const Problem pb, const Workspace ws) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t sQ = s_base + C::kOffQ, sRing = s_base + C::kOffRing, sP = s_base + C::kOffP;
+  const uint32_t bars = s_base + C::kOffBar;
+  auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffBar + 8 * kNumBars);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  int *status = ws.status;
+
+  // ---- work item: (b, h, query tile); causal runs the longest tiles first
+  const int nq = ws.nqb, bhq = pb.B * pb.Hq;
+  int qt, bh;
+  if (pb.is_causal) {
+    qt = nq - 1 - int(blockIdx.x / bhq);
+    bh = int(blockIdx.x % bhq);
+  } else {
+    qt = int(blockIdx.x % nq);
+    bh = int(blockIdx.x / nq);
+  }
+  const int b = bh / pb.Hq, h = bh % pb.Hq;
+  const int hk = h / (pb.Hq / pb.Hkv), bhk = b * pb.Hkv + hk;
+  const int q0 = qt * kQBlk;
+  const int nkt_all = ws.Nkv_pad / kKVTile;
+  int T = nkt_all;
+  if (pb.is_causal) T = min(nkt_all, min(q0 + kQBlk - 1, pb.Nq - 1) / kKVTile + 1);
+
+  if (threadIdx.x == 0) {
+    // the softmax warps (4) arrive on S-empty and P-full; TMA bytes or a
+    // single tcgen05.commit complete the others
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(bar(i), (i == kBarSEmpty || i == kBarPFull || i == kBarPFull + 1) ? 4 : 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip_all = *(volatile int *)status != 0;  // an earlier CTA already failed
+
+  if (warp == 0) {
+    // ================================================= TMA producer
+    if (lane == 0 && !skip_all) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
+      tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+      int n = 0;
+      bool ok = true;
+      auto issue = [&](bool isK, int j) {
+        if (!ok) return;
+        const int st = n % C::kStages;
+        const uint32_t ph = (n / C::kStages) & 1;
+        if (!mbar_wait(bar(kBarEmpty + st), ph ^ 1, status)) { ok = false; return; }
+        const uint32_t dst = sRing + st * C::kStageBytes;
+        if (isK) {
+          mbar_arrive_expect_tx(bar(kBarFull + st), C::kKBytes);
+          tma_load_2d(dst, &tm_k, bar(kBarFull + st), 0, bhk * ws.Nkv_pad + j * kKVTile);
+        } else {
+          mbar_arrive_expect_tx(bar(kBarFull + st), C::kVBytes);
+          tma_load_2d(dst, &tm_v, bar(kBarFull + st), j * kKVTile, bhk * D);
+        }
+        ++n;
+      };
+      issue(true, 0);
+      for (int j = 0; j < T; ++j) {
+        if (j + 1 < T) issue(true, j + 1);
+        issue(false, j);
+      }
+      // Before leaving, make sure every copy issued has landed (bounded).
+      mbar_wait(bar(kBarQ), 0, status, false);
+      for (int m = (n > C::kStages ? n - C::kStages : 0); m < n; ++m)
+        mbar_wait(bar(kBarFull + m % C::kStages), (m / C::kStages) & 1, status, false);
+    }
+  } else if (warp == 1) {
+    // ================================================= MMA issuer
+    if (lane == 0 && !skip_all) {
+      const uint32_t tS = tmem, tO = tmem + 128;
+      const uint32_t id_s = idesc_i8(128, 128);
+      const uint32_t id_o = idesc_e4m3_f32(128, D);
+      const uint64_t dQ = smem_desc_kmajor(sQ, C::Dp);
+      int n = 0;
+      bool ok = mbar_wait(bar(kBarQ), 0, status);
+      auto wait_stage = [&]() -> uint32_t {
+        const int st = n % C::kStages;
+        if (ok && !mbar_wait(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
+        return uint32_t(st);
+      };
+      auto issue_s = [&](uint32_t st) {
+        const uint64_t dK = smem_desc_kmajor(sRing + st * C::kStageBytes, C::Dp);
+#pragma unroll
+        for (int k = 0; k < C::kQKSteps; ++k)
+          mma_i8_ss(tS, dQ + 2 * k, dK + 2 * k, id_s, k > 0 ? 1u : 0u);
+        mma_commit(bar(kBarSFull));
+        mma_commit(bar(kBarEmpty + st));
+        ++n;
+      };
+      if (ok) {
+        const uint32_t st = wait_stage();
+        tc_fence_after();
+        if (ok) issue_s(st);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) {
+          const uint32_t st = wait_stage();
+          if (ok && !mbar_wait(bar(kBarSEmpty), j & 1, status)) ok = false;
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(st);
+        }
+        const uint32_t st = wait_stage();
+        if (ok && !mbar_wait(bar(kBarPFull + (j & 1)), (j >> 1) & 1, status)) ok = false;
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dP = smem_desc_kmajor(sP + (j & 1) * C::kPBytes, 128);
+        const uint64_t dV = smem_desc_kmajor(sRing + st * C::kStageBytes, 128);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_f8_ss(tO, dP + 2 * k, dV + 2 * k, id_o, (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(bar(kBarPVDone + (j & 1)));
+        mma_commit(bar(kBarEmpty + st));
+        ++n;
+      }
+      // every MMA issued by this thread has finished before teardown
+      mma_commit(bar(kBarFinal));
+      mbar_wait(bar(kBarFinal), 0, status, false);
+    }
+  } else {
+    // ================================================= softmax / correction / epilogue
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int row = 32 * wq + lane;          // row within the query tile
+    const int i = q0 + row;                  // query index
+    const uint32_t lane_off = uint32_t(32 * wq) << 16;
+    const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + 128;
+    const float qs = ws.q_scale[(long long)bh * nq + qt];
+    const float *ksc = ws.k_scale + (long long)bhk * (ws.Nkv_pad / kKBlk);
+    const float *dsk = kSmoothQ ? ws.dsk + ((long long)bh * nq + qt) * ws.Nkv_pad : nullptr;
+    float m_run = -INFINITY, l = 0.f;
+    bool ok = !skip_all;
+    for (int j = 0; ok && j < T; ++j) {
+      const int kb = j * kKVTile;
+      const float c0 = __fmul_rn(__fmul_rn(qs, ksc[2 * j]), pb.K2);
+      const float c1 = __fmul_rn(__fmul_rn(qs, ksc[2 * j + 1]), pb.K2);
+      if (!warp_wait(bar(kBarSFull), j & 1, status)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarSEmpty));
+
+      // valid keys of this tile for this row form the prefix [0, lim)
+      int lim = min(kKVTile, pb.Nkv - kb);
+      if (pb.is_causal) lim = min(lim, i - kb + 1);
+      const bool masked = lim < kKVTile;
+
+      float m_tile = -INFINITY;
+      if (!kSmoothQ) {
+        int mx0 = INT_MIN, mx1 = INT_MIN;
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (!masked || k < lim) mx0 = max(mx0, int(s[k]));
+#pragma unroll
+        for (int k = 64; k < 128; ++k)
+          if (!masked || k < lim) mx1 = max(mx1, int(s[k]));
+        if (mx0 != INT_MIN) m_tile = __fmul_rn(float(mx0), c0);
+        if (mx1 != INT_MIN) m_tile = fmaxf(m_tile, __fmul_rn(float(mx1), c1));
+      } else {
+#pragma unroll
+        for (int k = 0; k < 128; k += 4) {
+          const float4 d4 = __ldg(reinterpret_cast<const float4 *>(dsk + kb + k));
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            // s[] now holds the fp32 logits x = S * c + dS * K2
+            const float xv = __fmaf_rn(float(int(s[k + e])), k + e < 64 ? c0 : c1, dd[e]);
+            s[k + e] = __float_as_uint(xv);
+            if (!masked || k + e < lim) m_tile = fmaxf(m_tile, xv);
+          }
+        }
+      }
+      const float m_new = fmaxf(m_run, m_tile);
+      const float mb = (m_new == -INFINITY) ? 0.f : __fsub_rn(m_new, kLog2P8Max);
+      float alpha = 1.f;
+      if (m_run != m_new) alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(__fsub_rn(m_run, m_new));
+
+      uint32_t pk[32];
+      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+#pragma unroll
+      for (int k = 0; k < 128; k += 4) {
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float t = kSmoothQ ? __fsub_rn(__uint_as_float(s[k + e]), mb)
+                             : __fmaf_rn(float(int(s[k + e])), k + e < 64 ? c0 : c1, -mb);
+          if (masked && k + e >= lim) t = -INFINITY;
+          p[e] = ex2_approx(t);
+        }
+        ls0 += p[0];
+        ls1 += p[1];
+        ls2 += p[2];
+        ls3 += p[3];
+        pk[k / 4] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
+      }
+      l = __fmaf_rn(l, alpha, (ls0 + ls1) + (ls2 + ls3));
+
+      // P_j -> shared buffer j & 1, once P V_{j-2} has finished reading it
+      if (j >= 2 && !warp_wait(bar(kBarPVDone + (j & 1)), ((j - 2) >> 1) & 1, status)) {
+        ok = false;
+        break;
+      }
+      uint8_t *pbuf = smem + C::kOffP + (j & 1) * C::kPBytes;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4 *>(pbuf + swz_offset(row, 16 * cc, 128)) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+      fence_proxy_async_smem();
+
+      // rescale this row of O when the max grew (after P V_{j-1} is done)
+      const bool need = j > 0 && alpha != 1.f && m_run != -INFINITY;
+      if (__any_sync(0xffffffffu, need)) {
+        if (!warp_wait(bar(kBarPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + 32 * c, r);
+          if (need)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(tO + 32 * c, r);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(kBarPFull + (j & 1)));
+      m_run = m_new;
+    }
+
+    // ---- epilogue: out = O * v_scale / l (+ mean_v)
+    if (ok && warp_wait(bar(kBarPVDone + ((T - 1) & 1)), ((T - 1) >> 1) & 1, status)) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      const float *vs = ws.v_scale + (long long)bhk * D;
+      const float *mv = ws.mean_v + (long long)bhk * D;
+      uint8_t *orow = reinterpret_cast<uint8_t *>(pb.out) +
+                      2 * (b * pb.os_b + h * pb.os_h + (long long)i * pb.os_n);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + 32 * c, r);
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float o0 = __uint_as_float(r[e]) * (__ldg(vs + 32 * c + e) * inv_l);
+          float o1 = __uint_as_float(r[e + 1]) * (__ldg(vs + 32 * c + e + 1) * inv_l);
+          if (pb.smooth_v) {
+            o0 += __ldg(mv + 32 * c + e);
+            o1 += __ldg(mv + 32 * c + e + 1);
+          }
+          if (pb.bf16) {
+            const __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
+            packed[e / 2] = *reinterpret_cast<const uint32_t *>(&v2);
+          } else {
+            const __half2 v2 = __floats2half2_rn(o0, o1);
+            packed[e / 2] = *reinterpret_cast<const uint32_t *>(&v2);
+          }
+        }
+        if (i < pb.Nq) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            *reinterpret_cast<uint4 *>(orow + 64 * c + 16 * v4) =
+                make_uint4(packed[4 * v4], packed[4 * v4 + 1], packed[4 * v4 + 2], packed[4 * v4 + 3]);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------ debug: one S tile
+// 128 threads.  S = q8[qtile] k8[ktile]^T through TMA + tcgen05 kind::i8.
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+dump_s_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+              const Problem pb, const Workspace ws, int b, int h, int qtile, int ktile,
+              int32_t *s_out) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sQ = smem_u32(smem), sK = sQ + C::kQBytes;
+  const uint32_t bar0 = sK + C::kKBytes, bar1 = bar0 + 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kQBytes + C::kKBytes + 16);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar1, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int hk = h / (pb.Hq / pb.Hkv);
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar0, C::kQBytes + C::kKBytes);
+    tma_load_2d(sQ, &tm_q, bar0, 0, (b * pb.Hq + h) * ws.Nq_pad + qtile * 128);
+    tma_load_2d(sK, &tm_k, bar0, 0, (b * pb.Hkv + hk) * ws.Nkv_pad + ktile * 128);
+    ok = mbar_wait(bar0, 0, ws.status);
+    if (ok) {
+      tc_fence_after();
+      const uint64_t dQ = smem_desc_kmajor(sQ, C::Dp), dK = smem_desc_kmajor(sK, C::Dp);
+      for (int k = 0; k < C::kQKSteps; ++k)
+        mma_i8_ss(tmem, dQ + 2 * k, dK + 2 * k, idesc_i8(128, 128), k > 0 ? 1u : 0u);
+      mma_commit(bar1);
+    }
+  }
+  if (__syncthreads_and(ok ? 1 : 0) && warp_wait(bar1, 0, ws.status)) {
+    tc_fence_after();
+    const int row = 32 * warp + lane;
+    for (int c = 0; c < 4; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + 32 * c, r);
+      for (int e = 0; e < 32; ++e) s_out[row * 128 + 32 * c + e] = int32_t(r[e]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------ debug: one P V tile
+// 128 threads; P from global (row-major 128x128 e4m3) written into shared
+// memory with the kernel's swizzle; V tile by TMA; O = P V (kind::f8f6f4).
+template <int D>
+__global__ void __launch_bounds__(128, 1)
+debug_pv_kernel(const __grid_constant__ CUtensorMap tm_v, const Problem pb, const Workspace ws,
+                int b, int hkv, int ktile, const uint8_t *p8, float *o_out) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sP = smem_u32(smem), sV = sP + C::kPBytes;
+  const uint32_t bar0 = sV + C::kVBytes, bar1 = bar0 + 8;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kPBytes + C::kVBytes + 16);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int row = threadIdx.x;
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    mbar_init(bar1, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  for (int cc = 0; cc < 8; ++cc)
+    *reinterpret_cast<uint4 *>(smem + swz_offset(row, 16 * cc, 128)) =
+        *reinterpret_cast<const uint4 *>(p8 + row * 128 + 16 * cc);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar0, C::kVBytes);
+    tma_load_2d(sV, &tm_v, bar0, ktile * 128, (b * pb.Hkv + hkv) * D);
+    ok = mbar_wait(bar0, 0, ws.status);
+    if (ok) {
+      tc_fence_after();
+      const uint64_t dP = smem_desc_kmajor(sP, 128), dV = smem_desc_kmajor(sV, 128);
+      for (int k = 0; k < 4; ++k)
+        mma_f8_ss(tmem, dP + 2 * k, dV + 2 * k, idesc_e4m3_f32(128, D), k > 0 ? 1u : 0u);
+      mma_commit(bar1);
+    }
+  }
+  if (__syncthreads_and(ok ? 1 : 0) && warp_wait(bar1, 0, ws.status)) {
+    tc_fence_after();
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t r[32];
+      tmem_ld32(tmem + (uint32_t(32 * warp) << 16) + 32 * c, r);
+      for (int e = 0; e < 32; ++e) o_out[row * D + 32 * c + e] = __uint_as_float(r[e]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------ debug: e4m3
+__global__ void debug_e4m3_kernel(const float *in, uint8_t *out, int64_t n) {
+  const int64_t i = 2 * (int64_t(blockIdx.x) * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float lo = in[i], hi = (i + 1 < n) ? in[i + 1] : 0.f;
+  const uint32_t pr = e4m3x2(lo, hi);
+  out[i] = uint8_t(pr & 0xFF);
+  if (i + 1 < n) out[i + 1] = uint8_t(pr >> 8);
+}
+
+// ------------------------------------------------------------ debug: MMA loop
+// Back-to-back INT8 MMAs 128x256x32 from resident shared-memory operands.
+__global__ void __launch_bounds__(128, 1) mma_loop_kernel(int iters, int32_t *sink, int *status) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = align1024(smem_raw);
+  const uint32_t sA = smem_u32(smem), sB = sA + 128 * 128;
+  const uint32_t bar0 = sB + 256 * 128;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 128 * 128 + 256 * 128 + 16);
+  const int warp = threadIdx.x / 32;
+  for (int o = 4 * threadIdx.x; o < 384 * 128; o += 4 * blockDim.x)
+    *reinterpret_cast<uint32_t *>(smem + o) = 0x01010101u * ((o >> 7) & 3);
+  if (threadIdx.x == 0) {
+    mbar_init(bar0, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) {
+    const uint64_t dA = smem_desc_kmajor(sA, 128), dB = smem_desc_kmajor(sB, 128);
+    const uint32_t id = idesc_i8(128, 256);
+    for (int it = 0; it < iters; ++it)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mma_i8_ss(tmem, dA + 2 * k, dB + 2 * k, id, (it | k) ? 1u : 0u);
+    mma_commit(bar0);
+    mbar_wait(bar0, 0, status);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    uint32_t r[32];
+    tmem_ld32(tmem, r);
+    if (threadIdx.x == 0) sink[blockIdx.x] = int32_t(r[0]);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D, bool SQ>
+cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
+                                const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
+  using C = Cfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = unsigned(pb.B) * unsigned(pb.Hq) * unsigned(ws.nqb);
+  attn_fwd_kernel<D, SQ><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ debug: bounded wait
+__global__ void wait_timeout_kernel(int *status) {
+  __shared__ __align__(8) uint64_t b;
+  const uint32_t bar = smem_u32(&b);
+  mbar_init(bar, 1);
+  fence_mbar_init();
+  mbar_wait(bar, 0, status, false);  // nothing arrives: gives up after the limit
+}
+
+template <int D>
+cudaError_t launch_attention_d(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
+                               const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
+  return pb.smooth_q ? launch_attention_dq<D, true>(pb, ws, tq, tk, tv, stream)
+                     : launch_attention_dq<D, false>(pb, ws, tq, tk, tv, stream);
+}
+
+template <int D>
+cudaError_t launch_dump_s_d(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
+                            const CUtensorMap &tk, int b, int h, int qt, int kt, int32_t *s,
+                            cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int smem = C::kQBytes + C::kKBytes + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(dump_s_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dump_s_kernel<D><<<1, 128, smem, stream>>>(tq, tk, pb, ws, b, h, qt, kt, s);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_debug_pv_d(const Problem &pb, const Workspace &ws, const CUtensorMap &tv, int b,
+                              int hkv, int kt, const uint8_t *p8, float *o, cudaStream_t stream) {
+  using C = Cfg<D>;
+  const int smem = C::kPBytes + C::kVBytes + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(debug_pv_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  debug_pv_kernel<D><<<1, 128, smem, stream>>>(tv, pb, ws, b, hkv, kt, p8, o);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
+                             const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
+  switch (pb.D) {
+    case 64: return launch_attention_d<64>(pb, ws, tq, tk, tv, stream);
+    case 96: return launch_attention_d<96>(pb, ws, tq, tk, tv, stream);
+    case 128: return launch_attention_d<128>(pb, ws, tq, tk, tv, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_dump_s(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
+                          const CUtensorMap &tk, int b, int h, int qt, int kt, int32_t *s,
+                          cudaStream_t stream) {
+  switch (pb.D) {
+    case 64: return launch_dump_s_d<64>(pb, ws, tq, tk, b, h, qt, kt, s, stream);
+    case 96: return launch_dump_s_d<96>(pb, ws, tq, tk, b, h, qt, kt, s, stream);
+    case 128: return launch_dump_s_d<128>(pb, ws, tq, tk, b, h, qt, kt, s, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_debug_pv(const Problem &pb, const Workspace &ws, const CUtensorMap &tv, int b,
+                            int hkv, int kt, const uint8_t *p8, float *o, cudaStream_t stream) {
+  switch (pb.D) {
+    case 64: return launch_debug_pv_d<64>(pb, ws, tv, b, hkv, kt, p8, o, stream);
+    case 96: return launch_debug_pv_d<96>(pb, ws, tv, b, hkv, kt, p8, o, stream);
+    case 128: return launch_debug_pv_d<128>(pb, ws, tv, b, hkv, kt, p8, o, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_debug_e4m3(const float *in, uint8_t *out, int64_t n, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t pairs = (n + 1) / 2;
+  debug_e4m3_kernel<<<unsigned((pairs + 255) / 256), 256, 0, stream>>>(in, out, n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout(int *status, cudaStream_t stream) {
+  wait_timeout_kernel<<<1, 1, 0, stream>>>(status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mma_loop(int ctas, int iters, int32_t *sink, cudaStream_t stream) {
+  const int smem = 384 * 128 + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(mma_loop_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem);
+  if (e != cudaSuccess) return e;
+  // the sink doubles as the status word location after the per-CTA outputs
+  mma_loop_kernel<<<ctas, 128, smem, stream>>>(iters, sink, reinterpret_cast<int *>(sink + ctas));
+  return cudaGetLastError();
+}
+
+}  // namespace sage

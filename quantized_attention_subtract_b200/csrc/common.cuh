@@ -1,0 +1,68 @@
+// common.cuh -- constants and kernel parameter blocks of the CUDA path.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace sage {
+
+// Quantisation granularity and tiling.  The SageAttention pages fix
+// "per-block" quantisation of Q and K without block sizes ("sageattention"
+// package page, "What it is"); the reading taken: 128-token Q blocks (one
+// tensor-core M tile), 64-token K blocks (two per 128-key tile).
+constexpr int kQBlk = 128;
+constexpr int kKBlk = 64;
+constexpr int kKVTile = 128;
+
+// P is quantised as e4m3(448 * exp2(s - m)); 448 is e4m3's largest finite
+// value, so the row maximum maps to the top code.  log2(448) rounded to fp32.
+constexpr float kLog2P8Max = 8.80735492706298828125f;   // 0x410CEAED
+constexpr float kLog2e = 1.44269502162933349609375f;    // fp32(log2 e), 0x3FB8AA3B
+
+// Fixed-point means: sum of rint(x * 2^24) in int64.
+constexpr float kFixScale = 16777216.0f;
+
+// Workspace sub-buffers (device pointers), derived on the host.
+struct Workspace {
+  int8_t *q8;
+  int8_t *k8;
+  uint8_t *v8t;
+  float *q_scale, *k_scale, *v_scale;
+  float *mean_k, *mean_v;
+  float *mq, *dsk;
+  long long *k_sum, *v_sum;      // fixed-point channel sums [B*Hkv][D]
+  unsigned *v_max, *v_min;       // order-preserving keys of V channel max/min
+  int *status;
+  int Dp, Nq_pad, Nkv_pad, nqb, nkb;
+};
+
+// Shapes / flags / strides of one call, as the kernels see them.
+struct Problem {
+  const uint16_t *q, *k, *v;
+  void *out;
+  int B, Hq, Hkv, Nq, Nkv, D;
+  // element strides of (batch, head, token) for each tensor; the channel
+  // stride is 1
+  long long qs_b, qs_h, qs_n, ks_b, ks_h, ks_n, vs_b, vs_h, vs_n, os_b, os_h, os_n;
+  int bf16;
+  int is_causal, smooth_k, smooth_q, smooth_v;
+  float sm_scale;
+  float K2;  // fp32(sm_scale * fp32(log2 e))
+};
+
+// Host-side launchers (defined in prepass.cu / attn_fwd.cu).
+cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t stream);
+cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
+                             const CUtensorMap &tm_k, const CUtensorMap &tm_v, cudaStream_t stream);
+cudaError_t launch_dump_s(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
+                          const CUtensorMap &tm_k, int b, int h, int qtile, int ktile,
+                          int32_t *s_out, cudaStream_t stream);
+cudaError_t launch_debug_pv(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_v,
+                            int b, int hkv, int ktile, const uint8_t *p8, float *o_out,
+                            cudaStream_t stream);
+cudaError_t launch_debug_e4m3(const float *in, uint8_t *out, int64_t n, cudaStream_t stream);
+cudaError_t launch_mma_loop(int ctas, int iters, int32_t *sink, cudaStream_t stream);
+cudaError_t launch_wait_timeout(int *status, cudaStream_t stream);
+
+}  // namespace sage

@@ -1,0 +1,120 @@
+"""The C ABI library: loads without a GPU, exports every declared symbol, and
+rejects out-of-contract arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from quantized_attention_subtract_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sage_b200.h")
+GOLDEN = os.path.join(ROOT, "tests", "golden", "api_contract.txt")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^[a-z_0-9 \*]+?\b(sage_[a-z_0-9]+)\(", text, re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = binding.lib()
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(binding.EXPORTED) == names
+    assert L.sage_abi_version() == 1
+
+
+def test_status_strings():
+    L = binding.lib()
+    for code, name in binding.STATUS_NAMES.items():
+        assert L.sage_status_string(code).decode() == name
+
+
+def _params(**kw):
+    p = binding.Params()
+    d = dict(B=1, Hq=2, Hkv=2, Nq=256, Nkv=256, D=64, layout=0, dtype=0, is_causal=0, smooth_k=1)
+    d.update(kw)
+    for k, v in d.items():
+        setattr(p, k, v)
+    for name in ("q_strides", "k_strides", "v_strides", "o_strides"):
+        getattr(p, name)[:] = [d["Hq"] * d["Nq"] * d["D"], d["Nq"] * d["D"], d["D"], 1]
+    return p
+
+
+def _ws_size(p):
+    n = ctypes.c_size_t(0)
+    return binding.lib().sage_workspace_size(ctypes.byref(p), ctypes.byref(n)), n.value
+
+
+def _contract():
+    facts = {}
+    for line in open(GOLDEN):
+        if line.strip() and not line.startswith("#"):
+            key, *vals = line.split()
+            facts[key] = vals
+    return facts
+
+
+def test_head_dims_follow_the_pages():
+    allowed = {int(x) for x in _contract()["head_dims"]}
+    for D in range(16, 257, 16):
+        code, _ = _ws_size(_params(D=D))
+        assert (code == 0) == (D in allowed), D
+    assert _ws_size(_params(D=96))[0] == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hq=6, Hkv=4), 1), (dict(Nkv=0), 1), (dict(B=0), 1), (dict(Nq=-1), 1),
+    (dict(layout=2), 1), (dict(dtype=5), 2), (dict(is_causal=2), 1), (dict(D=80), 2),
+])
+def test_bad_shapes_rejected(kw, code):
+    assert _ws_size(_params(**kw))[0] == code
+
+
+def test_workspace_size_grows_with_smooth_q():
+    base = _ws_size(_params())[1]
+    withq = _ws_size(_params(smooth_q=1))[1]
+    assert withq > base > 0
+
+
+def _fwd(p):
+    return binding.lib().sage_attn_fwd(ctypes.byref(p), None)
+
+
+def test_argument_errors_before_any_device_work():
+    p = _params()
+    fake = 1 << 40  # never dereferenced: validation fails first
+    p.q = p.k = p.v = p.out = fake
+    p.workspace, p.workspace_bytes = fake, _ws_size(p)[1]
+    bad = _params()
+    bad.q = bad.k = bad.v = bad.out = fake + 8  # not 16-byte aligned
+    bad.workspace, bad.workspace_bytes = fake, p.workspace_bytes
+    assert _fwd(bad) == 3
+    p2 = _params()
+    p2.q = p2.k = p2.v = p2.out = fake
+    p2.q_strides[2] = 68  # token stride not a multiple of 8 elements
+    p2.workspace, p2.workspace_bytes = fake, p.workspace_bytes
+    assert _fwd(p2) == 3
+    p3 = _params()
+    p3.q = p3.k = p3.v = p3.out = fake
+    p3.workspace, p3.workspace_bytes = fake, p.workspace_bytes - 1
+    assert _fwd(p3) == 6
+    p4 = _params()
+    p4.q = p4.k = p4.v = p4.out = fake
+    p4.workspace, p4.workspace_bytes = fake + 128, p.workspace_bytes
+    assert _fwd(p4) == 6
+    p5 = _params()
+    p5.q = None
+    p5.workspace, p5.workspace_bytes = fake, p.workspace_bytes
+    assert _fwd(p5) == 1
+
+
+def test_binding_raises_without_the_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(binding, "_lib", None)
+    with pytest.raises(RuntimeError, match="CUDA library missing"):
+        binding.lib()
