@@ -63,41 +63,51 @@ def _oracle_problem(w: Workload):
                           smooth_q=w.smooth_q, smooth_v=w.smooth_v)
 
 
-def oracle_sample(w: Workload, kv_heads: int):
+def oracle_sample(w: Workload, kv_heads: int, q_tiles: int | None = None):
     """Time the CPU oracle (pre-pass + tiled attention) on the first `kv_heads`
-    kv heads of batch 0 with all their query heads and tiles.  Returns
-    (tops, seconds, description, threads)."""
+    kv heads of batch 0 with all their query heads, on the first `q_tiles`
+    query tiles of each (all when None).  Returns (tops, seconds, description,
+    threads)."""
     import oracle
     group = w.Hq // w.Hkv
     sub = w.with_(B=1, Hkv=kv_heads, Hq=kv_heads * group)
     q, k, v = generate(sub)
     pr = _oracle_problem(sub)
+    tiles = oracle.all_tiles(pr)
+    nt = pr.nqb if q_tiles is None else max(1, min(q_tiles, pr.nqb))
+    tiles = tiles[tiles[:, 2] < nt]
     t0 = time.perf_counter()
     pre = oracle.prepass(pr, q, k, v)
-    oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))
+    oracle.attention_tiles(pr, pre, tiles)
     dt = time.perf_counter() - t0
-    desc = (f"batch 0, kv heads 0..{kv_heads - 1} ({sub.Hq} query heads, all {pr.nqb} query tiles "
-            f"each) of {w.name}: pre-pass + tiled quantised attention")
-    return sub.ops / dt / 1e12, dt, desc, oracle.num_threads()
+    rows = sum(min(128, w.Nq - 128 * int(t)) for t in tiles[:, 2])
+    ops = 4.0 * rows * w.Nkv * w.D * (0.5 if w.is_causal else 1.0)
+    desc = (f"batch 0, kv heads 0..{kv_heads - 1} ({sub.Hq} query heads, query tiles 0..{nt - 1} "
+            f"each) of {w.name}: pre-pass of those heads + tiled quantised attention")
+    return ops / dt / 1e12, dt, desc, oracle.num_threads()
 
 
-def _sample_heads(w: Workload, target_s: float) -> int:
-    """kv heads of batch 0 whose oracle run takes about target_s seconds."""
-    import oracle
-    per_head = None
+def _sample_size(w: Workload, target_s: float):
+    """(kv_heads, q_tiles) of batch 0 whose oracle run takes about target_s seconds."""
     try:
-        _, dt, _, _ = oracle_sample(w.with_(Nq=min(w.Nq, 256)), 1)
-        per_head = dt * (w.Nq / min(w.Nq, 256))
+        _, dt, _, _ = oracle_sample(w, 1, 2)
+        per_tile = dt / (2 * (w.Hq // w.Hkv))
     except Exception:
-        per_head = 1.0
-    n = max(1, int(target_s / max(per_head, 1e-3)))
-    return min(n, w.Hkv)
+        per_tile = 0.05
+    tiles_total = max(1, int(target_s / max(per_tile, 1e-4)))
+    nqb = (w.Nq + 127) // 128
+    group = w.Hq // w.Hkv
+    per_head = nqb * group
+    if tiles_total >= per_head:
+        return min(w.Hkv, tiles_total // per_head), None
+    return 1, max(1, tiles_total // group)
 
 
 class ClockSampler:
-    """nvidia-smi SM clock / throttle-reason samples during the timed region."""
+    """nvidia-smi SM clock / throttle-reason samples; summary() keeps the
+    samples whose timestamps fall inside the marked timed region."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -105,19 +115,27 @@ class ClockSampler:
         self.gpu = gpu_index
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(1.0)  # let the sampler start before the timed region
         except Exception:
             self.proc = None
-        return self
 
-    def __exit__(self, *exc):
+    def mark_begin(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
+    def stop(self):
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -128,20 +146,30 @@ class ClockSampler:
     def summary(self):
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        from datetime import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) >= 9:
-                rows.append(parts)
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                continue
+            rows.append((ts, parts))
         os.unlink(self.path)
-        if not rows:
+        inside = [p for ts, p in rows if self.t0 is not None and self.t0 - 0.1 <= ts <= self.t1 + 0.1]
+        use = inside if inside else [p for _, p in rows]
+        if not use:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        num = lambda s: float(s) if s.replace(".", "", 1).isdigit() else None
+        sm = [num(r[2]) for r in use if num(r[2]) is not None]
+        mx = [num(r[3]) for r in use if num(r[3]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        reasons = sorted({names[i] for r in use for i in range(4) if r[6 + i].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(use),
+                "window": "timed region" if inside else "whole run (timed region shorter than one sample)"}
 
 
 def run_reference(args, w: Workload):
@@ -149,13 +177,15 @@ def run_reference(args, w: Workload):
     world, rank, _ = _dist()
     if rank != 0:
         return
-    heads = _sample_heads(w, 2.0)
+    # each step a bounded sample, so the whole run stays near two minutes
+    per_step = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    heads, tiles = _sample_size(w, per_step)
     for _ in range(args.warmup):
-        oracle_sample(w, heads)
+        oracle_sample(w, heads, tiles)
     times, tops = [], []
     desc, threads = "", 1
     for _ in range(args.steps):
-        t, dt, desc, threads = oracle_sample(w, heads)
+        t, dt, desc, threads = oracle_sample(w, heads, tiles)
         times.append(dt)
         tops.append(t)
     value = float(np.mean(tops))
@@ -204,33 +234,37 @@ def run_ours(args, w: Workload):
         torch.cuda.synchronize(dev)
 
     # ---- warm-up, then K timed steps of the whole pass
+    clk = ClockSampler(local)
+    clk.start()
     for _ in range(args.warmup):
         binding.attn_fwd(p, dev)
     barrier()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clk:
-        start.record(stream)
-        for _ in range(args.steps):
-            binding.attn_fwd(p, dev)
-        end.record(stream)
-        barrier()
-        step_ms = start.elapsed_time(end) / args.steps
-        # ---- the attention kernel alone (dominant kernel), per-launch events
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        for a, b in evs:
-            a.record(stream)
-            binding.attn_quantized(p, dev)
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-        # ---- the pre-pass alone
-        for a, b in evs:
-            a.record(stream)
-            binding.quantize(p, dev)
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        pre_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    clk.mark_begin()
+    start.record(stream)
+    for _ in range(args.steps):
+        binding.attn_fwd(p, dev)
+    end.record(stream)
+    barrier()
+    clk.mark_end()
+    step_ms = start.elapsed_time(end) / args.steps
+    # ---- the attention kernel alone (dominant kernel), per-launch events
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for a, b in evs:
+        a.record(stream)
+        binding.attn_quantized(p, dev)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    # ---- the pre-pass alone
+    for a, b in evs:
+        a.record(stream)
+        binding.quantize(p, dev)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    pre_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    clk.stop()
     clocks = clk.summary()
     assert binding.device_status(p) == 0, "device status nonzero"
 
@@ -284,8 +318,8 @@ def run_ours(args, w: Workload):
         "gpu_launches": kernels_per_step * args.steps,
     }
     if rank == 0 and not args.no_cpu_baseline:
-        heads = _sample_heads(w, 12.0)
-        tops, dt, desc, threads = oracle_sample(w, heads)
+        heads, tiles = _sample_size(w, 12.0)
+        tops, dt, desc, threads = oracle_sample(w, heads, tiles)
         line["cpu_baseline"] = {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
                                 "sample": desc + f" ({dt:.1f} s)"}
     if pg is not None:
@@ -298,8 +332,8 @@ def run_ours(args, w: Workload):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")

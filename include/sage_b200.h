@@ -74,6 +74,7 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
  * base pointer must be a multiple of 16 bytes (8 elements); tensors may not
  * overlap `out`.  Query head h reads kv head h / (Hq / Hkv); Hq % Hkv == 0.
  * D is 64, 96 or 128.  Nq >= 0, Nkv >= 1 (when Nq > 0); B, Hq, Hkv >= 1.
+ * With Nq == 0 the compute calls return SAGE_OK without reading any pointer.
  * is_causal masks key j for query i when j > i (top-left alignment, as in
  * scaled_dot_product_attention).  sm_scale <= 0 selects 1/sqrt(D).
  * The workspace holds the quantised tensors, scales and means; its size

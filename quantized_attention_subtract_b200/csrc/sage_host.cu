@@ -257,14 +257,18 @@ sage_status_t validate(const sage_attn_params_t *p, bool need_inputs, bool need_
 }
 
 sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, bool attn) {
+  // No queries: nothing to compute and no pointer is read (empty tensors
+  // may have null data pointers).
+  sage_status_t s = check_shape(p);
+  if (s != SAGE_OK) return s;
+  if (p->Nq == 0) return SAGE_OK;
   Layout L;
-  sage_status_t s = validate(p, pre, attn, L);
+  s = validate(p, pre, attn, L);
   if (s != SAGE_OK) return s;
   const Workspace ws = make_workspace(p, L);
   const Problem pb = make_problem(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (pre && cudaMemsetAsync(ws.status, 0, sizeof(int), st) != cudaSuccess) return SAGE_ERR_CUDA;
-  if (p->Nq == 0) return SAGE_OK;
   if (pre && launch_prepass(pb, ws, st) != cudaSuccess) return SAGE_ERR_CUDA;
   if (attn) {
     Maps m;
