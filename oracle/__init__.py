@@ -60,7 +60,7 @@ def _load():
             P = ctypes.POINTER(_Params)
             vp = ctypes.c_void_p
             lib.oracle_prepass.argtypes = [P] + [vp] * 13
-            lib.oracle_attention_tiles.argtypes = [P] + [vp] * 9 + [ctypes.c_int, vp, vp]
+            lib.oracle_attention_tiles.argtypes = [P] + [vp] * 9 + [ctypes.c_int, vp, vp, vp]
             lib.oracle_exact_attention_tiles.argtypes = [P, vp, vp, vp, ctypes.c_int, vp, vp]
             lib.oracle_round_output.argtypes = [P, vp, vp, ctypes.c_int64]
             lib.oracle_e4m3_encode_array.argtypes = [vp, vp, ctypes.c_int64]
@@ -158,19 +158,24 @@ def all_tiles(pr: Problem) -> np.ndarray:
                     np.int32).reshape(-1, 3)
 
 
-def attention_tiles(pr: Problem, pre: dict, tiles) -> np.ndarray:
+def attention_tiles(pr: Problem, pre: dict, tiles, with_uncertainty: bool = False):
     """Mirror of the tiled quantised attention for (b, h, q_tile) triples.
 
-    Returns fp64 [n_tiles, 128, D]; rows past Nq are zero.
+    Returns fp64 [n_tiles, 128, D] (rows past Nq are zero); with
+    `with_uncertainty`, also the per-element bound of how far an
+    implementation may differ because an FP8 code of P sits within the exp2
+    error band of an e4m3 rounding midpoint (see sage_oracle.c).
     """
     lib = _load()
     tiles = np.ascontiguousarray(np.asarray(tiles, np.int32).reshape(-1, 3))
     out = np.zeros((len(tiles), QBLK, pr.D), np.float64)
+    unc = np.zeros_like(out) if with_uncertainty else None
     c = pr._c()
     names = ("q8", "q_scale", "k8", "k_scale", "v8", "v_scale", "mean_v", "mq", "kp")
     lib.oracle_attention_tiles(ctypes.byref(c), *[_ptr(pre[n]) for n in names],
-                               len(tiles), _ptr(tiles), _ptr(out))
-    return out
+                               len(tiles), _ptr(tiles), _ptr(out),
+                               _ptr(unc) if unc is not None else None)
+    return (out, unc) if with_uncertainty else out
 
 
 def exact_attention_tiles(pr: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray, tiles) -> np.ndarray:

@@ -325,11 +325,24 @@ void oracle_delta_s(const oracle_params *p, const float *mq_blk, const float *kp
  * l (fp64) accumulates p, O (fp64) accumulates decode(P8) * decode(v8),
  * and both are multiplied by 2^(m_old - m_new) when the max grows.
  * Output o = O * v_scale / l (+ mean_v).
+ *
+ * unc (optional, same shape as out): how far an implementation may lie from
+ * `out` because the FP8 code of P is not unique.  The logit t is fixed to the
+ * bit by the steps above, but the pages fix no exp2 implementation; a fast
+ * hardware exp2 has a relative error of about 2^-22, so wherever 2^t lies
+ * within a relative band EXP2_BAND of an e4m3 rounding midpoint, both
+ * neighbouring codes are valid.  unc accumulates, per output channel, the
+ * effect of taking the other code: |step| * |v8| * v_scale / l.  With
+ * smoothed Q the correction dS enters t in fp32 on a GPU (fp64 here), so the
+ * band widens to EXP2_BAND_SMOOTH_Q.
  * ------------------------------------------------------------------- */
+#define EXP2_BAND 0x1p-19
+#define EXP2_BAND_SMOOTH_Q 0x1p-12
 void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const float *q_scale,
                             const int8_t *k8, const float *k_scale, const uint8_t *v8,
                             const float *v_scale, const float *mean_v, const float *mq,
-                            const float *kp, int n_tiles, const int *tiles, double *out) {
+                            const float *kp, int n_tiles, const int *tiles, double *out,
+                            double *unc) {
     const int D = p->D, Nq = p->Nq, Nkv = p->Nkv;
     const int nqb = (Nq + QBLK - 1) / QBLK, nkb = (Nkv + KBLK - 1) / KBLK;
     const int nkt = (Nkv + KVT - 1) / KVT;
@@ -352,6 +365,8 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
             const uint8_t *vh = v8 + ((int64_t)b * p->Hkv + hk) * Nkv * D;
             const float *ksh = k_scale + ((int64_t)b * p->Hkv + hk) * nkb;
             double *O = (double *)calloc((size_t)D, sizeof(double));
+            double *U = (double *)calloc((size_t)D, sizeof(double));
+            const double band = p->smooth_q ? EXP2_BAND_SMOOTH_Q : EXP2_BAND;
             double *dS = NULL;
             if (p->smooth_q) {
                 dS = (double *)malloc(sizeof(double) * (size_t)Nkv);
@@ -397,7 +412,10 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
                 double alpha = (m_run == -INFINITY) ? 0.0 : exp2((double)m_run - (double)m_new);
                 if (m_run != m_new) {
                     l *= alpha;
-                    for (int cc = 0; cc < D; cc++) O[cc] *= alpha;
+                    for (int cc = 0; cc < D; cc++) {
+                        O[cc] *= alpha;
+                        U[cc] *= alpha;
+                    }
                 }
                 for (int jj = 0; jj < KVT; jj++) {
                     if (!valid[jj]) continue;
@@ -408,9 +426,17 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
                     float pf = (float)exp2((double)tt);
                     if (pf < FLT_MIN) pf = 0.0f;
                     l += (double)pf;
-                    double pq = vdec[oracle_e4m3_encode((double)pf)];
+                    const uint8_t code = oracle_e4m3_encode((double)pf);
+                    double pq = vdec[code];
                     const uint8_t *vrow = vh + (int64_t)j * D;
                     for (int cc = 0; cc < D; cc++) O[cc] += pq * vdec[vrow[cc]];
+                    if (unc) {
+                        const double lo = vdec[oracle_e4m3_encode((double)pf * (1.0 - band))];
+                        const double hi = vdec[oracle_e4m3_encode((double)pf * (1.0 + band))];
+                        const double step = fmax(hi - pq, pq - lo);
+                        if (step > 0)
+                            for (int cc = 0; cc < D; cc++) U[cc] += step * fabs(vdec[vrow[cc]]);
+                    }
                 }
                 m_run = m_new;
             }
@@ -420,8 +446,10 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
             for (int cc = 0; cc < D; cc++) {
                 o[cc] = O[cc] * (double)vs[cc] / l;
                 if (p->smooth_v) o[cc] += (double)mv[cc];
+                if (unc) unc[((int64_t)t * QBLK + r) * D + cc] = U[cc] * (double)vs[cc] / l;
             }
             free(O);
+            free(U);
             free(dS);
         }
 }

@@ -103,15 +103,23 @@ def valid_rows(pr: oracle.Problem, tiles) -> np.ndarray:
 
 
 def compare_output(pr: oracle.Problem, pre: dict, q, k, v, g: GpuRun, tiles, exact: bool = True):
-    mirror = oracle.attention_tiles(pr, pre, tiles)
+    """GPU output vs the mirror (and vs exact fp64 attention) on `tiles`.
+
+    max_abs_excess is max(|gpu - mirror| - unc): the part of the difference
+    not explained by FP8 codes of P that the exp2 rounding leaves ambiguous
+    (both neighbouring codes valid; see the oracle's unc output)."""
+    mirror, unc = oracle.attention_tiles(pr, pre, tiles, with_uncertainty=True)
     got = oracle.tile_rows(pr, tiles, g.out_f64())
     rows = valid_rows(pr, tiles)
-    a, m = got[rows], mirror[rows]
-    res = dict(max_abs=float(np.max(np.abs(a - m))),
+    a, m, u = got[rows], mirror[rows], unc[rows]
+    d = np.abs(a - m)
+    res = dict(max_abs=float(d.max()), max_abs_excess=float(np.max(d - u)),
+               ambiguous_outputs=int((u > 0).sum()),
                cos=float((a * m).sum() / np.linalg.norm(a) / np.linalg.norm(m)))
     if exact:
         e = oracle.exact_attention_tiles(pr, q, k, v, tiles)[rows]
         res["rel_l1_exact"] = float(np.abs(a - e).sum() / np.abs(e).sum())
         res["cos_exact"] = float((a * e).sum() / np.linalg.norm(a) / np.linalg.norm(e))
         res["mirror_rel_l1_exact"] = float(np.abs(m - e).sum() / np.abs(e).sum())
+        res["mirror_cos_exact"] = float((m * e).sum() / np.linalg.norm(m) / np.linalg.norm(e))
     return res

@@ -1,5 +1,6 @@
 """GPU attention vs the oracle's mirror of the quantised algorithm (max |diff|
-<= 2e-2, cosine >= 0.9999) and vs exact fp64 attention (relative L1 <= 0.06,
+<= 2e-2 beyond the effect of FP8 codes of P that exp2 rounding leaves
+ambiguous, cosine >= 0.9999) and vs exact fp64 attention (relative L1 <= 0.06,
 cosine >= 0.998), every query tile of small problems spanning several tiles,
 ragged tails, both layouts, GQA, causal masking, all head dims and flags,
 plus the degenerate shapes."""
@@ -37,7 +38,7 @@ def test_attention_matches_oracle(case):
                        seed=11, k_offset_sigma=5.0, **flags)
     q, k, v, pr, pre, g = run_both(w)
     r = compare_output(pr, pre, q, k, v, g, oracle.all_tiles(pr))
-    assert r["max_abs"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
+    assert r["max_abs_excess"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
     assert r["rel_l1_exact"] <= EXACT_REL_L1 and r["cos_exact"] >= EXACT_COS, r
 
 

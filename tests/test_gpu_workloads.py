@@ -3,13 +3,17 @@ benchmark times (one sage_attn_fwd call on the default stream).
 
 Pre-pass outputs are compared bit for bit over the whole tensors; the output
 is compared on sampled query tiles (first, last/ragged and random ones) that
-the oracle computes row by row.  Against the mirror: max |diff| <= 2e-2 and
-cosine >= 0.9999.  Against exact fp64 attention: relative L1 <= 0.06 and
-cosine >= 0.998, except the workload whose Q/K/V carry x20 channel outliers,
-where per-block INT8 scales of Q and K are dominated by the outlier channels
-and the method itself (the oracle's mirror, not only the GPU) sits near 0.04
-relative L1 / 0.996 cosine; there the bound is relative L1 <= 0.06 and
-cosine >= 0.99.
+the oracle computes row by row.
+
+Against the mirror: max |diff| <= 2e-2 beyond the effect of FP8 codes of P
+that the exp2 rounding leaves ambiguous (the oracle's `unc`), and cosine >=
+0.9999.  Against exact fp64 attention the GPU must be no worse than the
+method itself (the mirror's own error, +0.002 relative L1 / -0.0005 cosine),
+and within an absolute bound per kind of input: iid inputs 0.06 / 0.998;
+x20 channel outliers in Q/K/V 0.06 / 0.99 (per-block INT8 scales of Q and K
+are dominated by the outlier channels); 2% of tokens x10 0.16 / 0.975 (almost
+every 128-token Q block and 64-token K block holds an outlier token, which
+sets its INT8 scale; the mirror alone measures 0.142 / 0.981 there).
 """
 import json
 import os
@@ -39,8 +43,13 @@ def test_workload_full_size(name, smooth_k):
     if report:
         with open(report, "a") as f:
             f.write(json.dumps(dict(workload=name, smooth_k=w.smooth_k, **r)) + "\n")
-    assert r["max_abs"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
+    assert r["max_abs_excess"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
+    assert r["rel_l1_exact"] <= r["mirror_rel_l1_exact"] + 0.002, r
+    assert r["cos_exact"] >= r["mirror_cos_exact"] - 0.0005, r
     if w.outlier_channels:
-        assert r["rel_l1_exact"] <= 0.06 and r["cos_exact"] >= 0.99, r
+        bound = (0.06, 0.99)
+    elif w.token_outlier_prob > 0:
+        bound = (0.16, 0.975)
     else:
-        assert r["rel_l1_exact"] <= EXACT_REL_L1 and r["cos_exact"] >= EXACT_COS, r
+        bound = (EXACT_REL_L1, EXACT_COS)
+    assert r["rel_l1_exact"] <= bound[0] and r["cos_exact"] >= bound[1], r

@@ -248,3 +248,21 @@ def test_mirror_is_layout_invariant():
     b = oracle.attention_tiles(pr_n, oracle.prepass(pr_n, *generate(w.with_(layout="NHD"))),
                                oracle.all_tiles(pr_n))
     assert np.array_equal(a, b)
+
+
+def test_uncertainty_is_zero_when_p_codes_are_exact_and_small_otherwise():
+    # Q = 0: every P equals 448 exactly, so no code is ambiguous.
+    w = random_problem(1, 2, 2, 256, 300, 64, dtype="fp16", seed=15)
+    pr = _problem(w)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, np.zeros_like(q), k, v)
+    _, unc = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr), with_uncertainty=True)
+    assert np.all(unc == 0)
+    # random inputs: a few ambiguous codes, each worth at most one e4m3 step
+    pre = oracle.prepass(pr, q, k, v)
+    out, unc = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr), with_uncertainty=True)
+    assert np.all(unc >= 0)
+    assert 0 < (unc > 0).mean() < 0.05
+    assert unc.max() < 0.05 * np.abs(out).max()
+    # the mirror itself is unchanged by asking for the bound
+    assert np.array_equal(out, oracle.attention_tiles(pr, pre, oracle.all_tiles(pr)))
