@@ -35,9 +35,13 @@
  *     independent of summation order.
  *   - V is FP8 e4m3 per channel over all tokens: scale = amax/448, code =
  *     e4m3_rn_satfinite(x * (448/amax)).
- *   - P is quantised as e4m3(448 * exp2(s - m)) (P <= 1 under the running
- *     max maps onto the full e4m3 range); the row sum l accumulates the
- *     unquantised values; O accumulates the quantised ones.
+ *   - Online softmax keeps, per row, a reference max m that is raised to a
+ *     tile's max only when that exceeds m by more than one binade (fp32
+ *     test t_max > m + 1); O and l are rescaled by 2^(m_old - m_new) only
+ *     then.  Every logit of a tile that did not raise m is <= m + 1, so P is
+ *     quantised as e4m3(224 * 2^(s - m)), which never exceeds 448 (e4m3's
+ *     largest finite value).  The row sum l accumulates the unquantised
+ *     values; O accumulates the quantised ones.
  *   - Causal masking is top-left aligned (key j is visible to query i when
  *     j <= i), as in scaled_dot_product_attention.
  *   - Query head h reads kv head h / (Hq / Hkv).
@@ -319,11 +323,12 @@ void oracle_delta_s(const oracle_params *p, const float *mq_blk, const float *kp
  * (rows >= Nq are left untouched).  S is formed in int64 from the codes;
  * per 128-key tile the row logits are s = S * c_half with
  * c_half = (q_scale * k_scale[half]) * K2, K2 = fl32(sm_scale * fl32(log2 e)),
- * all in fp32; the running max m and the shifted max mb = m - log2(448) are
- * fp32; the exponent is the fused fp32 t = S * c - mb; p = 2^t in fp64,
- * rounded to fp32 (flushing results below 2^-126 to zero); P8 = e4m3(p).
- * l (fp64) accumulates p, O (fp64) accumulates decode(P8) * decode(v8),
- * and both are multiplied by 2^(m_old - m_new) when the max grows.
+ * all in fp32; the reference max m (raised lazily, see above) and the
+ * shifted max mb = m - fl32(log2 224) are fp32; the exponent is the fused
+ * fp32 t = S * c - mb; p = 2^t in fp64, rounded to fp32 (flushing results
+ * below 2^-126 to zero); P8 = e4m3(p).  l (fp64) accumulates p, O (fp64)
+ * accumulates decode(P8) * decode(v8), and both are multiplied by
+ * 2^(m_old - m_new) when m is raised.
  * Output o = O * v_scale / l (+ mean_v).
  *
  * unc (optional, same shape as out): how far an implementation may lie from
@@ -348,7 +353,8 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
     const int nkt = (Nkv + KVT - 1) / KVT;
     const float log2e = 1.44269504088896340736f;
     const float K2 = p->sm_scale * log2e;
-    const float L448 = (float)log2(448.0);
+    const float LP = (float)log2(224.0);   /* P scale 224 = 448 / 2 */
+    const float LAZY = 1.0f;               /* raise m only past m + 1 */
     double vdec[256];
     for (int c = 0; c < 256; c++) vdec[c] = oracle_e4m3_decode((uint8_t)c);
 
@@ -407,16 +413,18 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
                     if (x[jj] > m_tile) m_tile = x[jj];
                 }
                 if (!any) continue;
-                float m_new = m_run > m_tile ? m_run : m_tile;
-                float mb = m_new - L448;
-                double alpha = (m_run == -INFINITY) ? 0.0 : exp2((double)m_run - (double)m_new);
-                if (m_run != m_new) {
-                    l *= alpha;
-                    for (int cc = 0; cc < D; cc++) {
-                        O[cc] *= alpha;
-                        U[cc] *= alpha;
+                if (m_run == -INFINITY || m_tile > m_run + LAZY) {
+                    if (m_run != -INFINITY) {
+                        const double alpha = exp2((double)m_run - (double)m_tile);
+                        l *= alpha;
+                        for (int cc = 0; cc < D; cc++) {
+                            O[cc] *= alpha;
+                            U[cc] *= alpha;
+                        }
                     }
+                    m_run = m_tile;
                 }
+                float mb = m_run - LP;
                 for (int jj = 0; jj < KVT; jj++) {
                     if (!valid[jj]) continue;
                     int j = kt * KVT + jj;
@@ -438,7 +446,6 @@ void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const floa
                             for (int cc = 0; cc < D; cc++) U[cc] += step * fabs(vdec[vrow[cc]]);
                     }
                 }
-                m_run = m_new;
             }
             double *o = out + ((int64_t)t * QBLK + r) * D;
             const float *vs = v_scale + ((int64_t)b * p->Hkv + hk) * D;

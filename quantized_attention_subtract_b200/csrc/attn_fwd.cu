@@ -73,6 +73,108 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int *st
   return __all_sync(0xffffffffu, ok);
 }
 
+// One query row's share of one KV tile (128 keys).  s[] holds the int32 S
+// row from TMEM; on return pk[] holds the 128 FP8 codes of P (key k in byte
+// k % 4 of pk[k / 4]) and lsum the sum of the unquantised probabilities.
+// m_used is the row's reference max (raised lazily, see kLazyLog2); alpha is
+// the factor O and l must be multiplied by (1 when m_used did not move).
+// Keys k >= lim are masked (only when kMasked).  Logits: x = S * c_half
+// (+ dsk with smoothed Q); the exponent t = x - (m_used - log2(224)) is one
+// fused fp32 op per key, as in the oracle.
+template <bool kMasked, bool kSmoothQ>
+__device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float c1,
+                                             const float *dsk_tile, int lim, float &m_used,
+                                             float &alpha, bool &rescale, float &lsum,
+                                             uint32_t (&pk)[32]) {
+  // s[] is converted in place: from here on it holds fp32 bit patterns,
+  // S as float (exact: |S| < 2^24), or the logits x with smoothed Q.
+#define X(k) __uint_as_float(s[k])
+#pragma unroll
+  for (int k = 0; k < 128; ++k) s[k] = __float_as_uint(__int2float_rn(int(s[k])));
+  if (kSmoothQ) {
+#pragma unroll
+    for (int k = 0; k < 128; k += 4) {
+      const float4 d4 = __ldg(reinterpret_cast<const float4 *>(dsk_tile + k));
+      const float c = k < 64 ? c0 : c1;
+      s[k] = __float_as_uint(__fmaf_rn(X(k), c, d4.x));
+      s[k + 1] = __float_as_uint(__fmaf_rn(X(k + 1), c, d4.y));
+      s[k + 2] = __float_as_uint(__fmaf_rn(X(k + 2), c, d4.z));
+      s[k + 3] = __float_as_uint(__fmaf_rn(X(k + 3), c, d4.w));
+    }
+  }
+  // ---- tile max over valid keys (per 64-key half before scaling)
+  float h0 = -INFINITY, h1 = -INFINITY, h2 = -INFINITY, h3 = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 64; k += 4) {
+    if (kMasked) {
+      h0 = fmax3(h0, k < lim ? X(k) : -INFINITY, k + 1 < lim ? X(k + 1) : -INFINITY);
+      h1 = fmax3(h1, k + 2 < lim ? X(k + 2) : -INFINITY, k + 3 < lim ? X(k + 3) : -INFINITY);
+      h2 = fmax3(h2, k + 64 < lim ? X(k + 64) : -INFINITY, k + 65 < lim ? X(k + 65) : -INFINITY);
+      h3 = fmax3(h3, k + 66 < lim ? X(k + 66) : -INFINITY, k + 67 < lim ? X(k + 67) : -INFINITY);
+    } else {
+      h0 = fmax3(h0, X(k), X(k + 1));
+      h1 = fmax3(h1, X(k + 2), X(k + 3));
+      h2 = fmax3(h2, X(k + 64), X(k + 65));
+      h3 = fmax3(h3, X(k + 66), X(k + 67));
+    }
+  }
+  const float lo = fmaxf(h0, h1), hi = fmaxf(h2, h3);
+  float m_tile;
+  if (kSmoothQ) {
+    m_tile = fmaxf(lo, hi);
+  } else {
+    // max_j fl(S_j * c) == fl(max_j S_j * c) since c >= 0
+    m_tile = fmaxf(lo == -INFINITY ? -INFINITY : __fmul_rn(lo, c0),
+                   hi == -INFINITY ? -INFINITY : __fmul_rn(hi, c1));
+  }
+  // ---- lazy reference max
+  alpha = 1.f;
+  rescale = false;
+  if (m_tile != -INFINITY && (m_used == -INFINITY || m_tile > __fadd_rn(m_used, kLazyLog2))) {
+    if (m_used != -INFINITY) {
+      alpha = ex2_approx(__fsub_rn(m_used, m_tile));
+      rescale = true;
+    } else {
+      alpha = 0.f;
+    }
+    m_used = m_tile;
+  }
+  const float nmb = m_used == -INFINITY ? 0.f : -__fsub_rn(m_used, kLog2P8Scale);
+  // ---- probabilities, their sum, FP8 codes
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 128; k += 4) {
+    float t0, t1, t2, t3;
+    if (kSmoothQ) {
+      t0 = __fadd_rn(X(k), nmb);
+      t1 = __fadd_rn(X(k + 1), nmb);
+      t2 = __fadd_rn(X(k + 2), nmb);
+      t3 = __fadd_rn(X(k + 3), nmb);
+    } else {
+      const float c = k < 64 ? c0 : c1;
+      t0 = __fmaf_rn(X(k), c, nmb);
+      t1 = __fmaf_rn(X(k + 1), c, nmb);
+      t2 = __fmaf_rn(X(k + 2), c, nmb);
+      t3 = __fmaf_rn(X(k + 3), c, nmb);
+    }
+    if (kMasked) {
+      t0 = k < lim ? t0 : -INFINITY;
+      t1 = k + 1 < lim ? t1 : -INFINITY;
+      t2 = k + 2 < lim ? t2 : -INFINITY;
+      t3 = k + 3 < lim ? t3 : -INFINITY;
+    }
+    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
+    const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
+    a0 += p0;
+    a1 += p1;
+    a2 += p2;
+    a3 += p3;
+    pk[k / 4] = e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
+  }
+  lsum = (a0 + a1) + (a2 + a3);
+#undef X
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -234,8 +336,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (!warp_wait(bar(kBarSFull), j & 1, status)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[128];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s + 32 * c);
+      tmem_ld128(tS, s);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarSEmpty));
@@ -243,57 +344,15 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // valid keys of this tile for this row form the prefix [0, lim)
       int lim = min(kKVTile, pb.Nkv - kb);
       if (pb.is_causal) lim = min(lim, i - kb + 1);
-      const bool masked = lim < kKVTile;
-
-      float m_tile = -INFINITY;
-      if (!kSmoothQ) {
-        int mx0 = INT_MIN, mx1 = INT_MIN;
-#pragma unroll
-        for (int k = 0; k < 64; ++k)
-          if (!masked || k < lim) mx0 = max(mx0, int(s[k]));
-#pragma unroll
-        for (int k = 64; k < 128; ++k)
-          if (!masked || k < lim) mx1 = max(mx1, int(s[k]));
-        if (mx0 != INT_MIN) m_tile = __fmul_rn(float(mx0), c0);
-        if (mx1 != INT_MIN) m_tile = fmaxf(m_tile, __fmul_rn(float(mx1), c1));
-      } else {
-#pragma unroll
-        for (int k = 0; k < 128; k += 4) {
-          const float4 d4 = __ldg(reinterpret_cast<const float4 *>(dsk + kb + k));
-          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            // s[] now holds the fp32 logits x = S * c + dS * K2
-            const float xv = __fmaf_rn(float(int(s[k + e])), k + e < 64 ? c0 : c1, dd[e]);
-            s[k + e] = __float_as_uint(xv);
-            if (!masked || k + e < lim) m_tile = fmaxf(m_tile, xv);
-          }
-        }
-      }
-      const float m_new = fmaxf(m_run, m_tile);
-      const float mb = (m_new == -INFINITY) ? 0.f : __fsub_rn(m_new, kLog2P8Max);
-      float alpha = 1.f;
-      if (m_run != m_new) alpha = (m_run == -INFINITY) ? 0.f : ex2_approx(__fsub_rn(m_run, m_new));
-
+      const float *dsk_tile = kSmoothQ ? dsk + kb : nullptr;
       uint32_t pk[32];
-      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
-#pragma unroll
-      for (int k = 0; k < 128; k += 4) {
-        float p[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float t = kSmoothQ ? __fsub_rn(__uint_as_float(s[k + e]), mb)
-                             : __fmaf_rn(float(int(s[k + e])), k + e < 64 ? c0 : c1, -mb);
-          if (masked && k + e >= lim) t = -INFINITY;
-          p[e] = ex2_approx(t);
-        }
-        ls0 += p[0];
-        ls1 += p[1];
-        ls2 += p[2];
-        ls3 += p[3];
-        pk[k / 4] = e4m3x2(p[0], p[1]) | (e4m3x2(p[2], p[3]) << 16);
-      }
-      l = __fmaf_rn(l, alpha, (ls0 + ls1) + (ls2 + ls3));
+      float alpha, lsum;
+      bool need;
+      if (lim >= kKVTile)
+        softmax_tile<false, kSmoothQ>(s, c0, c1, dsk_tile, lim, m_run, alpha, need, lsum, pk);
+      else
+        softmax_tile<true, kSmoothQ>(s, c0, c1, dsk_tile, lim, m_run, alpha, need, lsum, pk);
+      l = __fmaf_rn(l, alpha, lsum);
 
       // P_j -> shared buffer j & 1, once P V_{j-2} has finished reading it
       if (j >= 2 && !warp_wait(bar(kBarPVDone + (j & 1)), ((j - 2) >> 1) & 1, status)) {
@@ -307,8 +366,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       fence_proxy_async_smem();
 
-      // rescale this row of O when the max grew (after P V_{j-1} is done)
-      const bool need = j > 0 && alpha != 1.f && m_run != -INFINITY;
+      // rescale this row of O when its reference max moved (after P V_{j-1} is done)
       if (__any_sync(0xffffffffu, need)) {
         if (!warp_wait(bar(kBarPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, status)) {
           ok = false;
@@ -328,7 +386,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + (j & 1)));
-      m_run = m_new;
     }
 
     // ---- epilogue: out = O * v_scale / l (+ mean_v)

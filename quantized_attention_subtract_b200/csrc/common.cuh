@@ -15,9 +15,14 @@ constexpr int kQBlk = 128;
 constexpr int kKBlk = 64;
 constexpr int kKVTile = 128;
 
-// P is quantised as e4m3(448 * exp2(s - m)); 448 is e4m3's largest finite
-// value, so the row maximum maps to the top code.  log2(448) rounded to fp32.
-constexpr float kLog2P8Max = 8.80735492706298828125f;   // 0x410CEAED
+// Online softmax with a lazily raised reference max m: a row's m is raised
+// to the tile max only when that exceeds m by more than kLazyLog2 (one
+// binade); O and l are rescaled only then.  Every logit s of a tile that did
+// not raise m satisfies s <= m + 1, so P is quantised as
+// e4m3(224 * 2^(s - m)) <= e4m3(448), e4m3's largest finite value.
+// kLog2P8Scale = fp32(log2(224)).
+constexpr float kLazyLog2 = 1.0f;
+constexpr float kLog2P8Scale = 7.807354927062988281f;   // 0x40F9D5DA
 constexpr float kLog2e = 1.44269502162933349609375f;    // fp32(log2 e), 0x3FB8AA3B
 
 // Fixed-point means: sum of rint(x * 2^24) in int64.

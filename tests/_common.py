@@ -102,18 +102,32 @@ def valid_rows(pr: oracle.Problem, tiles) -> np.ndarray:
     return m
 
 
+def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Half a unit in the last place of the 16-bit output type at |x|: the
+    largest error of the final round-to-nearest store (bf16 keeps 8
+    significant bits, fp16 11; fp16 subnormals have a fixed 2^-24 step)."""
+    _, e = np.frexp(np.abs(x))          # |x| = f * 2^e, f in [0.5, 1)
+    bits = 8 if dtype == "bf16" else 11
+    h = np.ldexp(1.0, e - bits - 1)
+    if dtype == "fp16":
+        h = np.maximum(h, 2.0 ** -25)
+    return h
+
+
 def compare_output(pr: oracle.Problem, pre: dict, q, k, v, g: GpuRun, tiles, exact: bool = True):
     """GPU output vs the mirror (and vs exact fp64 attention) on `tiles`.
 
-    max_abs_excess is max(|gpu - mirror| - unc): the part of the difference
-    not explained by FP8 codes of P that the exp2 rounding leaves ambiguous
-    (both neighbouring codes valid; see the oracle's unc output)."""
+    max_abs_excess is max(|gpu - mirror| - unc - half_ulp): the part of the
+    difference explained neither by FP8 codes of P that the exp2 rounding
+    leaves ambiguous (both neighbouring codes valid; the oracle's unc output)
+    nor by the final rounding of the output to its 16-bit type."""
     mirror, unc = oracle.attention_tiles(pr, pre, tiles, with_uncertainty=True)
     got = oracle.tile_rows(pr, tiles, g.out_f64())
     rows = valid_rows(pr, tiles)
     a, m, u = got[rows], mirror[rows], unc[rows]
     d = np.abs(a - m)
-    res = dict(max_abs=float(d.max()), max_abs_excess=float(np.max(d - u)),
+    hu = half_ulp(np.maximum(np.abs(a), np.abs(m)), pr.dtype)
+    res = dict(max_abs=float(d.max()), max_abs_excess=float(np.max(d - u - hu)),
                ambiguous_outputs=int((u > 0).sum()),
                cos=float((a * m).sum() / np.linalg.norm(a) / np.linalg.norm(m)))
     if exact:

@@ -1,6 +1,6 @@
 """GPU attention vs the oracle's mirror of the quantised algorithm (max |diff|
 <= 2e-2 beyond the effect of FP8 codes of P that exp2 rounding leaves
-ambiguous, cosine >= 0.9999) and vs exact fp64 attention (relative L1 <= 0.06,
+ambiguous and half an ulp of the 16-bit output, cosine >= 0.9999) and vs exact fp64 attention (relative L1 <= 0.06,
 cosine >= 0.998), every query tile of small problems spanning several tiles,
 ragged tails, both layouts, GQA, causal masking, all head dims and flags,
 plus the degenerate shapes."""
