@@ -140,6 +140,29 @@ sage_status_t sage_quantize(const sage_attn_params_t *p, sage_stream_t stream);
  * the same parameters.  Writes p->out. */
 sage_status_t sage_attn_quantized(const sage_attn_params_t *p, sage_stream_t stream);
 
+/* sage_attn_fwd for callers that cannot allocate device memory.  Some hosts
+ * hand this library a fixed memory budget and forbid allocations once they
+ * have started (serving runtimes with pre-planned pools, plug-in hosts that
+ * own the device heap), and some call from latency-critical loops where a
+ * cudaMalloc would synchronise the device and stall the caller.  Those
+ * callers cannot provide the workspace.
+ * This entry point ignores p->workspace / p->workspace_bytes and uses a
+ * library-owned scratch area instead: a static device array of
+ * SAGE_NOALLOC_MAX_WORKSPACE_BYTES (64 MiB) that every GPU which loads this
+ * library holds until the process exits.  The caller still passes q, k, v and
+ * out.  Problems whose workspace (sage_workspace_size) exceeds that limit are
+ * rejected with SAGE_ERR_WORKSPACE before anything is enqueued.  The first
+ * call on each device looks up the array's device address (with that device
+ * current); make that first call before any stream capture.  Nothing here
+ * allocates.  All calls share the one array and it keeps the last call's
+ * contents; each call clears what must start at zero.  Calls that overlap on
+ * the GPU (other streams, other threads) race on the array and must be
+ * serialised by the caller.  sage_get_device_status does not see this
+ * array; a device timeout still makes later results unreliable.
+ * The SageAttention pages have no counterpart of this call. */
+#define SAGE_NOALLOC_MAX_WORKSPACE_BYTES (64ull << 20)
+sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t stream);
+
 /* Debug: the int32 tile S = q8 k8^T of query tile `qtile` (128 rows) and key
  * tile `ktile` (128 keys) of (batch b, query head h), computed by the same
  * tensor-core path as the attention kernel from a filled workspace, written

@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
 EXPORTED = ["sage_abi_version", "sage_status_string", "sage_workspace_size", "sage_workspace_view",
             "sage_attn_fwd", "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
             "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop", "sage_debug_wait_timeout",
-            "sage_get_device_status"]
+            "sage_get_device_status", "sage_attn_fwd_noalloc"]
 
 
 class SageError(RuntimeError):
@@ -79,7 +79,8 @@ def lib():
             L.sage_status_string.argtypes = [ctypes.c_int]
             L.sage_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
             L.sage_workspace_view.argtypes = [P, ctypes.POINTER(WorkspaceView)]
-            for f in (L.sage_attn_fwd, L.sage_quantize, L.sage_attn_quantized):
+            for f in (L.sage_attn_fwd, L.sage_quantize, L.sage_attn_quantized,
+                      L.sage_attn_fwd_noalloc):
                 f.argtypes = [P, vp]
             L.sage_debug_dump_s.argtypes = [P, i32, i32, i32, i32, vp, vp]
             L.sage_debug_pv.argtypes = [P, i32, i32, i32, vp, vp, vp]
@@ -90,7 +91,8 @@ def lib():
             for name in ("sage_workspace_size", "sage_workspace_view", "sage_attn_fwd",
                          "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
                          "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop",
-                         "sage_debug_wait_timeout", "sage_get_device_status"):
+                         "sage_debug_wait_timeout", "sage_get_device_status",
+                         "sage_attn_fwd_noalloc"):
                 getattr(L, name).restype = ctypes.c_int
             _lib = L
     return _lib
@@ -187,6 +189,16 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
         res.copy_(dev_out, non_blocking=True)
         return res
     return dev_out
+
+
+NOALLOC_MAX_WORKSPACE_BYTES = 64 << 20
+
+
+def attn_fwd_noalloc(p: Params, device) -> None:
+    """sage_attn_fwd on the library's own static scratch (p.workspace is
+    ignored); for callers that cannot allocate device memory on the call path.
+    Calls share that scratch: serialise them."""
+    _check(lib().sage_attn_fwd_noalloc(ctypes.byref(p), _stream(device)), "sage_attn_fwd_noalloc")
 
 
 def quantize(p: Params, device) -> None:

@@ -278,6 +278,31 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   return SAGE_OK;
 }
 
+// Library-owned scratch for sage_attn_fwd_noalloc (see the header): one
+// array per device that loads the library, alive until the process exits.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[SAGE_NOALLOC_MAX_WORKSPACE_BYTES];
+
+// Device address of g_noalloc_scratch per device ordinal, looked up once with
+// that device current.  In host code the array's name is only a host-side
+// stand-in, never a device address.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+sage_status_t noalloc_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SAGE_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SAGE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -331,6 +356,19 @@ sage_status_t sage_workspace_view(const sage_attn_params_t *p, sage_workspace_vi
 
 sage_status_t sage_attn_fwd(const sage_attn_params_t *p, sage_stream_t stream) {
   return run(p, stream, true, true);
+}
+
+sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t stream) {
+  sage_status_t s = check_shape(p);
+  if (s != SAGE_OK) return s;
+  if (make_layout(p).total > SAGE_NOALLOC_MAX_WORKSPACE_BYTES) return SAGE_ERR_WORKSPACE;
+  if ((s = check_device()) != SAGE_OK) return s;
+  void *scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != SAGE_OK) return s;
+  sage_attn_params_t q = *p;
+  q.workspace = scratch;
+  q.workspace_bytes = SAGE_NOALLOC_MAX_WORKSPACE_BYTES;
+  return run(&q, stream, true, true);
 }
 
 sage_status_t sage_quantize(const sage_attn_params_t *p, sage_stream_t stream) {
