@@ -102,22 +102,27 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float
       s[k + 3] = __float_as_uint(__fmaf_rn(X(k + 3), c, d4.w));
     }
   }
-  // ---- tile max over valid keys (per 64-key half before scaling)
-  float h0 = -INFINITY, h1 = -INFINITY, h2 = -INFINITY, h3 = -INFINITY;
+  // ---- tile max over valid keys (per 64-key half before scaling); eight
+  // independent 3-input max chains keep the dependency depth at 8
+  float h[8];
 #pragma unroll
-  for (int k = 0; k < 64; k += 4) {
-    if (kMasked) {
-      h0 = fmax3(h0, k < lim ? X(k) : -INFINITY, k + 1 < lim ? X(k + 1) : -INFINITY);
-      h1 = fmax3(h1, k + 2 < lim ? X(k + 2) : -INFINITY, k + 3 < lim ? X(k + 3) : -INFINITY);
-      h2 = fmax3(h2, k + 64 < lim ? X(k + 64) : -INFINITY, k + 65 < lim ? X(k + 65) : -INFINITY);
-      h3 = fmax3(h3, k + 66 < lim ? X(k + 66) : -INFINITY, k + 67 < lim ? X(k + 67) : -INFINITY);
-    } else {
-      h0 = fmax3(h0, X(k), X(k + 1));
-      h1 = fmax3(h1, X(k + 2), X(k + 3));
-      h2 = fmax3(h2, X(k + 64), X(k + 65));
-      h3 = fmax3(h3, X(k + 66), X(k + 67));
+  for (int q = 0; q < 8; ++q) h[q] = -INFINITY;
+#pragma unroll
+  for (int k = 0; k < 64; k += 8) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k0 = k + 2 * q, k1 = k0 + 64;
+      if (kMasked) {
+        h[q] = fmax3(h[q], k0 < lim ? X(k0) : -INFINITY, k0 + 1 < lim ? X(k0 + 1) : -INFINITY);
+        h[q + 4] = fmax3(h[q + 4], k1 < lim ? X(k1) : -INFINITY, k1 + 1 < lim ? X(k1 + 1) : -INFINITY);
+      } else {
+        h[q] = fmax3(h[q], X(k0), X(k0 + 1));
+        h[q + 4] = fmax3(h[q + 4], X(k1), X(k1 + 1));
+      }
     }
   }
+  const float h0 = fmaxf(h[0], h[1]), h1 = fmaxf(h[2], h[3]);
+  const float h2 = fmaxf(h[4], h[5]), h3 = fmaxf(h[6], h[7]);
   const float lo = fmaxf(h0, h1), hi = fmaxf(h2, h3);
   float m_tile;
   if (kSmoothQ) {
@@ -364,7 +369,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int cc = 0; cc < 8; ++cc)
         *reinterpret_cast<uint4 *>(pbuf + swz_offset(row, 16 * cc, 128)) =
             make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-      fence_proxy_async_smem();
 
       // rescale this row of O when its reference max moved (after P V_{j-1} is done)
       if (__any_sync(0xffffffffu, need)) {
@@ -373,16 +377,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           break;
         }
         tc_fence_after();
+        // the whole O row in one TMEM round trip
+        uint32_t r[D];
+        if constexpr (D == 128) {
+          tmem_ld128(tO, r);
+        } else if constexpr (D == 96) {
+          tmem_ld64(tO, r);
+          tmem_ld32(tO + 64, r + 64);
+        } else {
+          tmem_ld64(tO, r);
+        }
+        if (need)
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + 32 * c, r);
-          if (need)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tO + 32 * c, r);
+          for (int e = 0; e < D; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+        if constexpr (D == 128) {
+          tmem_st128(tO, r);
+        } else if constexpr (D == 96) {
+          tmem_st64(tO, r);
+          tmem_st32(tO + 64, r + 64);
+        } else {
+          tmem_st64(tO, r);
         }
       }
+      // P stores visible to the tensor core (async proxy), TMEM writes ordered,
+      // then P_j is handed to the MMA warp
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarPFull + (j & 1)));

@@ -10,15 +10,16 @@
 //   kv_stats   per (b, kv head, 256-token chunk): fixed-point channel sums of
 //              K (and V) and the V channel max/min, combined with atomics
 //              (integer addition is exact, so the order does not matter);
-//   quantize   per 128-token tile of Q, K or V: smoothing, block amax,
+//   quantize   per 128-token tile of K, V or Q (in that order, K/V heads in
+//              reverse so their second read hits L2): smoothing, block amax,
 //              INT8/FP8 codes written through shared memory as whole
 //              coalesced tiles in the attention kernel's layout (V
 //              transposed so that keys are contiguous);
 //   delta_s    (smooth_q only) the correction dS[blk][j] = mq[blk] . K'_j,
 //              stored pre-multiplied by sm_scale * log2(e).
 //
-// Every thread owns one 16-byte chunk (8 channels) of a row and walks rows
-// 16 apart, so loads are 16-byte vectors and a warp covers whole rows.
+// Threads own 16-byte chunks (8 channels) of rows, so loads are 16-byte
+// vectors and a warp covers whole rows.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -69,8 +70,10 @@ __device__ __forceinline__ long long fixed_point(float x) {
 }
 
 // ------------------------------------------------------------ kv_stats
-// grid (ceil(Nkv / 256), B * Hkv), block 16 * (D / 8)
-__global__ void kv_stats_kernel(Problem pb, Workspace ws) {
+// grid (ceil(Nkv / 256), B * Hkv), block 16 * (D / 8).  Each thread owns one
+// 16-byte chunk (8 channels) and walks rows 16 apart, two rows per step so
+// that four 16-byte loads are in flight before any arithmetic.
+__global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace ws) {
   const int C8 = pb.D / 8;
   const int c8 = threadIdx.x % C8, r0 = threadIdx.x / C8;
   const int bh = blockIdx.y, b = bh / pb.Hkv, h = bh % pb.Hkv;
@@ -87,21 +90,28 @@ __global__ void kv_stats_kernel(Problem pb, Workspace ws) {
     vmax[e] = -INFINITY;
     vmin[e] = INFINITY;
   }
-  for (int r = r0; r < kStatTokens; r += kRowsPerPass) {
-    const int j = j0 + r;
-    if (j >= pb.Nkv) break;
-    float x[8];
-    if (pb.smooth_k) {
-      load8(kb + j * pb.ks_n, pb.bf16, x);
+  for (int rr = r0; rr < kStatTokens; rr += 2 * kRowsPerPass) {
+    float xk[2][8], xv[2][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ksum[e] += fixed_point(x[e]);
+    for (int u = 0; u < 2; ++u) {
+      const int j = j0 + rr + u * kRowsPerPass;
+      if (j < pb.Nkv) {
+        if (pb.smooth_k) load8(kb + j * pb.ks_n, pb.bf16, xk[u]);
+        load8(vb + j * pb.vs_n, pb.bf16, xv[u]);
+      }
     }
-    load8(vb + j * pb.vs_n, pb.bf16, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      vmax[e] = fmaxf(vmax[e], x[e]);
-      vmin[e] = fminf(vmin[e], x[e]);
-      if (pb.smooth_v) vsum[e] += fixed_point(x[e]);
+    for (int u = 0; u < 2; ++u) {
+      const int j = j0 + rr + u * kRowsPerPass;
+      if (j < pb.Nkv) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (pb.smooth_k) ksum[e] += fixed_point(xk[u][e]);
+          vmax[e] = fmaxf(vmax[e], xv[u][e]);
+          vmin[e] = fminf(vmin[e], xv[u][e]);
+          if (pb.smooth_v) vsum[e] += fixed_point(xv[u][e]);
+        }
+      }
     }
   }
 
@@ -151,7 +161,8 @@ __global__ void kv_stats_kernel(Problem pb, Workspace ws) {
   }
 }
 
-// Block-wide max of two values (one per K half, or the same value twice).
+// Block-wide max of two values (one per K half, or the same value twice);
+// up to 32 warps.
 __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -173,10 +184,10 @@ __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
   }
 }
 
-__device__ __forceinline__ int8_t int8_code(float x, float inv) {
+__device__ __forceinline__ uint32_t int8_code(float x, float inv) {
   int q = __float2int_rn(__fmul_rn(x, inv));
   q = q > 127 ? 127 : (q < -127 ? -127 : q);
-  return int8_t(q);
+  return uint32_t(q) & 0xFFu;
 }
 
 // Copy a finished [rows][row_bytes] tile from shared memory to a contiguous
@@ -187,166 +198,94 @@ __device__ __forceinline__ void store_tile(uint8_t *dst, const uint8_t *src, int
 }
 
 // ------------------------------------------------------------ quantize
-// grid (nQ + nK + nV), block 16 * (D / 8).  Each CTA quantises one
-// 128-token tile: a Q block, a K tile (two 64-token blocks) or a V tile.
-__global__ void __launch_bounds__(256) quantize_kernel(Problem pb, Workspace ws) {
+// grid (nK + nV + nQ), block 32 * (D / 8): thread t owns channels
+// 8 * (t % (D/8)) .. +7 of the four consecutive rows 4 * (t / (D/8)) .. +3 of
+// one 128-token tile.  Block order: K and V tiles first, heads in reverse
+// order (those kv_stats read last are still in L2), then Q blocks.
+__global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws) {
   __shared__ __align__(16) uint8_t tile[128 * 128];
-  __shared__ long long red[kRowsPerPass][128];
+  __shared__ unsigned long long colsum[128];
   __shared__ float chan[128];
   __shared__ float scratch[64];
 
   const int D = pb.D, Dp = ws.Dp, C8 = D / 8;
-  const int c8 = threadIdx.x % C8, r0 = threadIdx.x / C8;
-  const int nQ = pb.B * pb.Hq * ws.nqb;
+  const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;  // rows 4 rg .. 4 rg + 3
   const int nKt = ws.Nkv_pad / kKVTile;
-  const int nK = pb.B * pb.Hkv * nKt;
+  const int nKV = pb.B * pb.Hkv * nKt;
   int blk = blockIdx.x;
+  float x[4][8];
 
-  float x[8][8];  // [row i][channel e]: row r0 + 16 i, channel 8 c8 + e
-
-  if (blk < nQ) {
-    // ---------------- Q block: optional block mean, INT8 per block
-    const int qb = blk % ws.nqb, bh = blk / ws.nqb, b = bh / pb.Hq, h = bh % pb.Hq;
-    const int i0 = qb * kQBlk, nvalid = min(kQBlk, pb.Nq - i0);
-    const uint16_t *src = pb.q + b * pb.qs_b + h * pb.qs_h + 8 * c8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
-      if (r < nvalid) load8(src + (long long)(i0 + r) * pb.qs_n, pb.bf16, x[i]);
-      else
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
-    }
-    if (pb.smooth_q) {
-      long long s[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (r0 + kRowsPerPass * i < nvalid)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) s[e] += fixed_point(x[i][e]);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) red[r0][8 * c8 + e] = s[e];
-      __syncthreads();
-      if (threadIdx.x < D) {
-        long long t = 0;
-        for (int r = 0; r < kRowsPerPass; ++r) t += red[r][threadIdx.x];
-        const float m = fixed_mean(t, nvalid);
-        chan[threadIdx.x] = m;
-        ws.mq[((long long)bh * ws.nqb + qb) * D + threadIdx.x] = m;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (r0 + kRowsPerPass * i < nvalid)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[i][e] = __fsub_rn(x[i][e], chan[8 * c8 + e]);
-    }
-    float a = 0.f, unused = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[i][e]));
-    block_max2(a, unused, scratch);
-    float inv = 0.f, scale = 0.f;
-    if (a >= kTinyAmax) {
-      scale = __fdiv_rn(a, 127.0f);
-      inv = __fdiv_rn(127.0f, a);
-    }
-    if (threadIdx.x == 0) ws.q_scale[(long long)bh * ws.nqb + qb] = scale;
-    // codes -> smem tile [128][Dp] (pad rows hold zeros since x == 0 there)
-    if (Dp != D)
-      for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
-        *reinterpret_cast<uint32_t *>(tile + o) = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w0 |= uint32_t(uint8_t(int8_code(x[i][e], inv))) << (8 * e);
-        w1 |= uint32_t(uint8_t(int8_code(x[i][e + 4], inv))) << (8 * e);
-      }
-      *reinterpret_cast<uint2 *>(tile + r * Dp + 8 * c8) = make_uint2(w0, w1);
-    }
-    __syncthreads();
-    store_tile(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)bh * ws.Nq_pad + i0) * Dp, tile,
-               128 * Dp);
-    return;
-  }
-  blk -= nQ;
-  if (blk < nK) {
-    // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
-    const int kt = blk % nKt, bh = blk / nKt, b = bh / pb.Hkv, h = bh % pb.Hkv;
+  if (blk < 2 * nKV) {
+    const int isV = blk & 1;
+    const int kvi = nKV - 1 - (blk >> 1);  // reverse head order
+    const int kt = kvi % nKt, bh = kvi / nKt, b = bh / pb.Hkv, h = bh % pb.Hkv;
     const int j0 = kt * kKVTile, nvalid = max(0, min(kKVTile, pb.Nkv - j0));
-    const uint16_t *src = pb.k + b * pb.ks_b + h * pb.ks_h + 8 * c8;
-    float mean[8];
+    if (!isV) {
+      // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
+      const uint16_t *src = pb.k + b * pb.ks_b + h * pb.ks_h + 8 * c8;
+      float mean[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-      mean[e] = pb.smooth_k ? fixed_mean(ws.k_sum[(long long)bh * D + 8 * c8 + e], pb.Nkv) : 0.f;
-    if (kt == 0 && r0 == 0)
+      for (int e = 0; e < 8; ++e)
+        mean[e] = pb.smooth_k ? fixed_mean(ws.k_sum[(long long)bh * D + 8 * c8 + e], pb.Nkv) : 0.f;
+      if (kt == 0 && rg == 0)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ws.mean_k[(long long)bh * D + 8 * c8 + e] = mean[e];
+        for (int e = 0; e < 8; ++e) ws.mean_k[(long long)bh * D + 8 * c8 + e] = mean[e];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
-      if (r < nvalid) {
-        load8(src + (long long)(j0 + r) * pb.ks_n, pb.bf16, x[i]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = __fsub_rn(x[i][e], mean[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+      for (int u = 0; u < 4; ++u) {
+        const int r = 4 * rg + u;
+        if (r < nvalid) load8(src + (long long)(j0 + r) * pb.ks_n, pb.bf16, x[u]);
       }
-    }
-    float a0 = 0.f, a1 = 0.f;  // rows 0..63 and 64..127
+      float a = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+      for (int u = 0; u < 4; ++u) {
+        if (4 * rg + u < nvalid) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (i < 4) a0 = fmaxf(a0, fabsf(x[i][e]));
-        else a1 = fmaxf(a1, fabsf(x[i][e]));
+          for (int e = 0; e < 8; ++e) {
+            x[u][e] = __fsub_rn(x[u][e], mean[e]);
+            a = fmaxf(a, fabsf(x[u][e]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
+        }
       }
-    block_max2(a0, a1, scratch);
-    float inv0 = 0.f, inv1 = 0.f, s0 = 0.f, s1 = 0.f;
-    if (a0 >= kTinyAmax) {
-      s0 = __fdiv_rn(a0, 127.0f);
-      inv0 = __fdiv_rn(127.0f, a0);
-    }
-    if (a1 >= kTinyAmax) {
-      s1 = __fdiv_rn(a1, 127.0f);
-      inv1 = __fdiv_rn(127.0f, a1);
-    }
-    if (threadIdx.x == 0) {
-      ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt] = s0;
-      ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt + 1] = s1;
-    }
-    if (Dp != D)
-      for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
-        *reinterpret_cast<uint32_t *>(tile + o) = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
-      const float inv = i < 4 ? inv0 : inv1;
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w0 |= uint32_t(uint8_t(int8_code(x[i][e], inv))) << (8 * e);
-        w1 |= uint32_t(uint8_t(int8_code(x[i][e + 4], inv))) << (8 * e);
+      // rows 0..63 belong to block 2 kt, rows 64..127 to 2 kt + 1
+      float a0 = rg < 16 ? a : 0.f, a1 = rg < 16 ? 0.f : a;
+      block_max2(a0, a1, scratch);
+      float inv0 = 0.f, inv1 = 0.f, s0 = 0.f, s1 = 0.f;
+      if (a0 >= kTinyAmax) {
+        s0 = __fdiv_rn(a0, 127.0f);
+        inv0 = __fdiv_rn(127.0f, a0);
       }
-      *reinterpret_cast<uint2 *>(tile + r * Dp + 8 * c8) = make_uint2(w0, w1);
+      if (a1 >= kTinyAmax) {
+        s1 = __fdiv_rn(a1, 127.0f);
+        inv1 = __fdiv_rn(127.0f, a1);
+      }
+      if (threadIdx.x == 0) {
+        ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt] = s0;
+        ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt + 1] = s1;
+      }
+      const float inv = rg < 16 ? inv0 : inv1;
+      if (Dp != D)
+        for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
+          *reinterpret_cast<uint32_t *>(tile + o) = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          w0 |= int8_code(x[u][e], inv) << (8 * e);
+          w1 |= int8_code(x[u][e + 4], inv) << (8 * e);
+        }
+        *reinterpret_cast<uint2 *>(tile + (4 * rg + u) * Dp + 8 * c8) = make_uint2(w0, w1);
+      }
+      __syncthreads();
+      store_tile(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)bh * ws.Nkv_pad + j0) * Dp, tile,
+                 128 * Dp);
+      return;
     }
-    __syncthreads();
-    store_tile(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)bh * ws.Nkv_pad + j0) * Dp, tile,
-               128 * Dp);
-    return;
-  }
-  blk -= nK;
-  {
     // ---------------- V tile: V' = V - mean_v, FP8 per channel, transposed
-    const int vt = blk % nKt, bh = blk / nKt, b = bh / pb.Hkv, h = bh % pb.Hkv;
-    const int j0 = vt * kKVTile, nvalid = max(0, min(kKVTile, pb.Nkv - j0));
     const uint16_t *src = pb.v + b * pb.vs_b + h * pb.vs_h + 8 * c8;
     float mean[8], inv[8];
 #pragma unroll
@@ -356,47 +295,128 @@ __global__ void __launch_bounds__(256) quantize_kernel(Problem pb, Workspace ws)
       const float hi = __fsub_rn(key_float(ws.v_max[ci]), mean[e]);
       const float lo = __fsub_rn(key_float(ws.v_min[ci]), mean[e]);
       const float a = fmaxf(fabsf(hi), fabsf(lo));
-      float s = 0.f;
+      float sc = 0.f;
       inv[e] = 0.f;
       if (a >= kTinyAmax) {
-        s = __fdiv_rn(a, 448.0f);
+        sc = __fdiv_rn(a, 448.0f);
         inv[e] = __fdiv_rn(448.0f, a);
       }
-      if (vt == 0 && r0 == 0) {
-        ws.v_scale[ci] = s;
+      if (kt == 0 && rg == 0) {
+        ws.v_scale[ci] = sc;
         ws.mean_v[ci] = mean[e];
       }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
+    for (int u = 0; u < 4; ++u) {
+      const int r = 4 * rg + u;
       if (r < nvalid) {
-        load8(src + (long long)(j0 + r) * pb.vs_n, pb.bf16, x[i]);
+        load8(src + (long long)(j0 + r) * pb.vs_n, pb.bf16, x[u]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = __fmul_rn(__fsub_rn(x[i][e], mean[e]), inv[e]);
+        for (int e = 0; e < 8; ++e) x[u][e] = __fmul_rn(__fsub_rn(x[u][e], mean[e]), inv[e]);
       } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = 0.f;
+        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
       }
     }
-    // transposed smem tile [D][128 keys]
+    // Transposed tile [D][128 keys] as 32 words per channel row; the word of
+    // keys 4 rg .. 4 rg + 3 of channel c sits at position (rg + rot * c8) % 32,
+    // which puts the 32 lanes of a warp on 32 different banks.
+    const int rot = 32 / (C8 == 12 ? 16 : C8);
+    uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = r0 + kRowsPerPass * i;
+    for (int e = 0; e < 8; e += 2) {
+      uint32_t w_lo = 0, w_hi = 0;
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        const uint32_t pr = e4m3x2(x[i][e], x[i][e + 1]);
-        tile[(8 * c8 + e) * 128 + r] = uint8_t(pr & 0xFF);
-        tile[(8 * c8 + e + 1) * 128 + r] = uint8_t(pr >> 8);
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t pr = e4m3x2(x[u][e], x[u][e + 1]);
+        w_lo |= (pr & 0xFFu) << (8 * u);
+        w_hi |= (pr >> 8) << (8 * u);
       }
+      const int pos = (rg + rot * c8) & 31;
+      tw[(8 * c8 + e) * 32 + pos] = w_lo;
+      tw[(8 * c8 + e + 1) * 32 + pos] = w_hi;
     }
     __syncthreads();
     uint8_t *dst = ws.v8t + (long long)bh * D * ws.Nkv_pad + j0;
-    for (int o = 16 * threadIdx.x; o < D * 128; o += 16 * blockDim.x) {
-      const int c = o / 128, k = o % 128;
-      *reinterpret_cast<uint4 *>(dst + (long long)c * ws.Nkv_pad + k) =
-          *reinterpret_cast<const uint4 *>(tile + o);
+    for (int t = threadIdx.x; t < D * 8; t += blockDim.x) {
+      const int c = t >> 3, q = t & 7;  // channel row c, keys 16 q .. 16 q + 15
+      const int sh = rot * (c >> 3);
+      uint4 o;
+      o.x = tw[c * 32 + ((4 * q + 0 + sh) & 31)];
+      o.y = tw[c * 32 + ((4 * q + 1 + sh) & 31)];
+      o.z = tw[c * 32 + ((4 * q + 2 + sh) & 31)];
+      o.w = tw[c * 32 + ((4 * q + 3 + sh) & 31)];
+      *reinterpret_cast<uint4 *>(dst + (long long)c * ws.Nkv_pad + 16 * q) = o;
     }
+    return;
+  }
+  blk -= 2 * nKV;
+  {
+    // ---------------- Q block: optional block mean, INT8 per block
+    const int qb = blk % ws.nqb, bh = blk / ws.nqb, b = bh / pb.Hq, h = bh % pb.Hq;
+    const int i0 = qb * kQBlk, nvalid = min(kQBlk, pb.Nq - i0);
+    const uint16_t *src = pb.q + b * pb.qs_b + h * pb.qs_h + 8 * c8;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = 4 * rg + u;
+      if (r < nvalid) load8(src + (long long)(i0 + r) * pb.qs_n, pb.bf16, x[u]);
+      else
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
+    }
+    if (pb.smooth_q) {
+      if (threadIdx.x < D) colsum[threadIdx.x] = 0ull;
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        long long s = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * rg + u < nvalid) s += fixed_point(x[u][e]);
+        atomicAdd(&colsum[8 * c8 + e], (unsigned long long)s);
+      }
+      __syncthreads();
+      if (threadIdx.x < D) {
+        const float m = fixed_mean((long long)colsum[threadIdx.x], nvalid);
+        chan[threadIdx.x] = m;
+        ws.mq[((long long)bh * ws.nqb + qb) * D + threadIdx.x] = m;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (4 * rg + u < nvalid)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[u][e] = __fsub_rn(x[u][e], chan[8 * c8 + e]);
+    }
+    float a = 0.f, unused = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[u][e]));
+    block_max2(a, unused, scratch);
+    float inv = 0.f, scale = 0.f;
+    if (a >= kTinyAmax) {
+      scale = __fdiv_rn(a, 127.0f);
+      inv = __fdiv_rn(127.0f, a);
+    }
+    if (threadIdx.x == 0) ws.q_scale[(long long)bh * ws.nqb + qb] = scale;
+    if (Dp != D)
+      for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
+        *reinterpret_cast<uint32_t *>(tile + o) = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        w0 |= int8_code(x[u][e], inv) << (8 * e);
+        w1 |= int8_code(x[u][e + 4], inv) << (8 * e);
+      }
+      *reinterpret_cast<uint2 *>(tile + (4 * rg + u) * Dp + 8 * c8) = make_uint2(w0, w1);
+    }
+    __syncthreads();
+    store_tile(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)bh * ws.Nq_pad + i0) * Dp, tile,
+               128 * Dp);
   }
 }
 
@@ -453,14 +473,13 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(ws.v_min, 0xFF, nch * sizeof(unsigned), stream);
   if (e != cudaSuccess) return e;
-  const int threads = 16 * (pb.D / 8);
   dim3 g1((pb.Nkv + kStatTokens - 1) / kStatTokens, pb.B * pb.Hkv);
-  kv_stats_kernel<<<g1, threads, 0, stream>>>(pb, ws);
+  kv_stats_kernel<<<g1, 16 * (pb.D / 8), 0, stream>>>(pb, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int nKt = ws.Nkv_pad / kKVTile;
   const long long nblk = (long long)pb.B * pb.Hq * ws.nqb + 2LL * pb.B * pb.Hkv * nKt;
-  quantize_kernel<<<dim3((unsigned)nblk), threads, 0, stream>>>(pb, ws);
+  quantize_kernel<<<dim3((unsigned)nblk), 32 * (pb.D / 8), 0, stream>>>(pb, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pb.smooth_q) {
