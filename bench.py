@@ -39,6 +39,27 @@ METRIC = "attention TOPS (4*B*H*Nq*Nkv*d/s) at N=4K-32K, d=128; % of B200 tensor
 DEFAULT_WORKLOAD = "mha_n4096_d128_bf16"
 L2_BYTES = 126 * 1024 * 1024
 
+# DRAM bytes (read + write) per launch of the attention kernel on the default
+# workload, from one ncu capture (profiles/attn_fwd_kernel_mha_n4096_d128_bf16.md).
+# They describe the kernel built from the sources hashed here; after any change
+# to those sources the traffic is reported as null until it is captured again.
+ATTN_TRAFFIC = {"workload": DEFAULT_WORKLOAD, "sources_sha256_16": "bfc4eb11cb537a46", "bytes": 302737664}
+ATTN_SOURCES = ["attn_fwd.cu", "ptx.cuh", "common.cuh"]
+
+
+def _attn_traffic(w: Workload):
+    import hashlib
+    csrc = os.path.join(ROOT, "quantized_attention_subtract_b200", "csrc")
+    try:
+        data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ATTN_SOURCES)
+    except OSError:
+        return None
+    if w.name != ATTN_TRAFFIC["workload"]:
+        return None
+    if hashlib.sha256(data).hexdigest()[:16] != ATTN_TRAFFIC["sources_sha256_16"]:
+        return None
+    return ATTN_TRAFFIC["bytes"]
+
 
 def _peaks():
     try:
@@ -308,7 +329,7 @@ def run_ours(args, w: Workload):
                    "smooth_k": w.smooth_k, "parallelism": f"replicas x{world}",
                    "l2": f"inputs {in_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)"},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
-                     "peak": peak8, "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": None,
+                     "peak": peak8, "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": _attn_traffic(w),
                      "peak_source": f"{peak_src} bf16 x 2 (burst)", "attn_ms": attn_ms,
                      "prepass_ms": pre_ms,
                      "prepass_gbs": 3 * (qd.numel() + kd.numel() + vd.numel()) / (pre_ms * 1e-3) / 1e9},
