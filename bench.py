@@ -77,6 +77,22 @@ def _dist():
     return world, rank, local
 
 
+def max_over_ranks(values, dist=None, device="cpu"):
+    """Element-wise max of per-rank timings (every rank gets the result); with
+    no process group the values come back unchanged."""
+    if dist is None:
+        return [float(x) for x in values]
+    import torch
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def replica_value(world: int, ops_per_replica: float, ms: float) -> float:
+    """Whole-job TOPS of `world` independent replicas timed at `ms` (max over ranks)."""
+    return world * ops_per_replica / (ms * 1e-3) / 1e12
+
+
 def _oracle_problem(w: Workload):
     import oracle
     return oracle.Problem(B=w.B, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, Nkv=w.Nkv, D=w.D, layout=w.layout,
@@ -290,10 +306,7 @@ def run_ours(args, w: Workload):
     assert binding.device_status(p) == 0, "device status nonzero"
 
     # max over ranks
-    t = torch.tensor([step_ms, attn_ms, pre_ms], device=dev)
-    if pg is not None:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    step_ms, attn_ms, pre_ms = (float(x) for x in t.tolist())
+    step_ms, attn_ms, pre_ms = max_over_ranks([step_ms, attn_ms, pre_ms], pg, dev)
 
     # ---- end to end through the public API with pinned host buffers
     qh, kh, vh = (x.cpu().pin_memory() for x in (qd, kd, vd))
@@ -308,15 +321,12 @@ def run_ours(args, w: Workload):
         sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh)
     e1.record(stream)
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / e2e_steps], device=dev)
-    if pg is not None:
-        pg.all_reduce(e2e_ms, op=pg.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms, = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], pg, dev)
 
     bf16_tflops, hbm_gbs, peak_src = _peaks()
     peak8 = 2.0 * bf16_tflops  # 8-bit dense = 2 x bf16 dense (nominal 4.5 / 2.25 PFLOP/s)
     achieved = w.ops / (attn_ms * 1e-3) / 1e12
-    value = world * w.ops / (step_ms * 1e-3) / 1e12
+    value = replica_value(world, w.ops, step_ms)
     kernels_per_step = 3 + (1 if w.smooth_q else 0)  # kv_stats, quantize, (delta_s), attention
 
     line = {
@@ -333,7 +343,7 @@ def run_ours(args, w: Workload):
                      "peak_source": f"{peak_src} bf16 x 2 (burst)", "attn_ms": attn_ms,
                      "prepass_ms": pre_ms,
                      "prepass_gbs": 3 * (qd.numel() + kd.numel() + vd.numel()) / (pre_ms * 1e-3) / 1e9},
-        "e2e": {"value": world * w.ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        "e2e": {"value": replica_value(world, w.ops, e2e_ms), "unit": "TOPS",
                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * 2},
         "clocks": clocks,
         "gpu_launches": kernels_per_step * args.steps,

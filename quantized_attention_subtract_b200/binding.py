@@ -167,15 +167,19 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
     """Quantized attention forward: INT8 Q K^T, FP8 P V, on the current CUDA stream.
 
     q: [B, Hq, Nq, D] ("HND") or [B, Nq, Hq, D] ("NHD"); k, v: same with Hkv, Nkv.
-    Host (CPU) tensors are copied to the current device and the result back.
+    Host (CPU) tensors are moved to the current device and the result back, in
+    chunks of whole (batch, kv-head group) slices so that the host-to-device
+    copy of one chunk, the kernels of the previous one and the device-to-host
+    copy of the one before overlap; the returned host tensor is complete once
+    the current stream has passed this call (pinned host tensors make the
+    copies asynchronous).
     """
-    host = not q.is_cuda
-    if host:
-        dev = torch.device("cuda", torch.cuda.current_device())
-        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
-    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+    if not q.is_cuda:
+        return _sageattn_host(q, k, v, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
+                              smooth_v, out)
+    if not (k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be on the same device")
-    dev_out = torch.empty_like(q) if (out is None or host) else out
+    dev_out = torch.empty_like(q) if out is None else out
     p = make_params(q, k, v, dev_out, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
                     smooth_v)
     if workspace is None:
@@ -183,12 +187,84 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
     else:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
     _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(q.device)), "sage_attn_fwd")
-    if host:
-        res = out if out is not None else torch.empty(dev_out.shape, dtype=dev_out.dtype,
-                                                      pin_memory=True)
-        res.copy_(dev_out, non_blocking=True)
-        return res
     return dev_out
+
+
+# Copy/compute pipelining of host-tensor calls: at least this many bytes of
+# inputs per chunk, at most this many chunks.
+_HOST_CHUNK_MIN_BYTES = 8 << 20
+_HOST_MAX_CHUNKS = 16
+
+
+def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int):
+    """Split (batch, kv head) into contiguous slices [(b, h0, h1)] of whole kv heads."""
+    total = B * Hkv
+    n = max(1, min(_HOST_MAX_CHUNKS, total, (total * bytes_per_kv_head) // _HOST_CHUNK_MIN_BYTES))
+    per_batch = -(-n // B)                       # chunks per batch entry
+    per_b = -(-Hkv // per_batch)                 # kv heads per chunk
+    chunks = []
+    for b in range(B):
+        for h0 in range(0, Hkv, per_b):
+            chunks.append((b, h0, min(Hkv, h0 + per_b)))
+    return chunks
+
+
+def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    B, Hq, Nq, D = _dims(q, layout)
+    _, Hkv, Nkv, _ = _dims(k, layout)
+    group = Hq // Hkv if Hkv else 1
+    res = out if out is not None else torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    hq_axis = 1 if layout == "HND" else 2
+    # whole-problem device buffers; each chunk is a (batch, head-range) view
+    qd, kd, vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (q, k, v))
+    od = torch.empty(q.shape, dtype=q.dtype, device=dev)
+    per_kv = (k.element_size() * Nkv * D * 2 + q.element_size() * group * Nq * D * 2)
+    chunks = _host_chunks(B, Hkv, group, per_kv)
+
+    def sl(t, b, h0, h1):
+        idx = [slice(b, b + 1), slice(None), slice(None), slice(None)]
+        idx[hq_axis] = slice(h0, h1)
+        return t[tuple(idx)]
+
+    compute = torch.cuda.current_stream(dev)
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d.wait_stream(compute)
+    first = make_params(sl(qd, *chunks[0][:1], chunks[0][1] * group, chunks[0][2] * group),
+                        sl(kd, *chunks[0]), sl(vd, *chunks[0]),
+                        sl(od, chunks[0][0], chunks[0][1] * group, chunks[0][2] * group),
+                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+    ws = alloc_workspace(first, dev)
+    done_out = None
+    for b, h0, h1 in chunks:
+        qh, kh, vh = sl(q, b, h0 * group, h1 * group), sl(k, b, h0, h1), sl(v, b, h0, h1)
+        qc, kc, vc = sl(qd, b, h0 * group, h1 * group), sl(kd, b, h0, h1), sl(vd, b, h0, h1)
+        oc, ohost = sl(od, b, h0 * group, h1 * group), sl(res, b, h0 * group, h1 * group)
+        with torch.cuda.stream(h2d):
+            qc.copy_(qh, non_blocking=True)
+            kc.copy_(kh, non_blocking=True)
+            vc.copy_(vh, non_blocking=True)
+            landed = torch.cuda.Event()
+            landed.record(h2d)
+        compute.wait_event(landed)
+        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+        need = workspace_bytes(p)
+        if need > ws.numel():
+            ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+        _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(dev)), "sage_attn_fwd")
+        computed = torch.cuda.Event()
+        computed.record(compute)
+        d2h.wait_event(computed)
+        with torch.cuda.stream(d2h):
+            ohost.copy_(oc, non_blocking=True)
+            done_out = torch.cuda.Event()
+            done_out.record(d2h)
+    compute.wait_event(done_out)
+    # keep the device buffers alive until the queued work has used them
+    for t in (qd, kd, vd, od, ws):
+        t.record_stream(compute)
+    return res
 
 
 NOALLOC_MAX_WORKSPACE_BYTES = 64 << 20

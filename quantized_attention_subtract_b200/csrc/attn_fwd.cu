@@ -87,10 +87,10 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float
                                              float &alpha, bool &rescale, float &lsum,
                                              uint32_t (&pk)[32]) {
   // s[] is converted in place: from here on it holds fp32 bit patterns,
-  // S as float (exact: |S| < 2^24), or the logits x with smoothed Q.
+  // S as float (exact), or the logits x with smoothed Q.
 #define X(k) __uint_as_float(s[k])
 #pragma unroll
-  for (int k = 0; k < 128; ++k) s[k] = __float_as_uint(__int2float_rn(int(s[k])));
+  for (int k = 0; k < 128; ++k) s[k] = __float_as_uint(s32_to_f32_exact(s[k]));
   if (kSmoothQ) {
 #pragma unroll
     for (int k = 0; k < 128; k += 4) {
@@ -174,7 +174,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float
     a1 += p1;
     a2 += p2;
     a3 += p3;
-    pk[k / 4] = e4m3x2(p0, p1) | (e4m3x2(p2, p3) << 16);
+    pk[k / 4] = e4m3x4(p0, p1, p2, p3);
   }
   lsum = (a0 + a1) + (a2 + a3);
 #undef X

@@ -35,6 +35,7 @@ struct Workspace {
   uint8_t *v8t;
   float *q_scale, *k_scale, *v_scale;
   float *mean_k, *mean_v;
+  float *v_inv;                  // 448 / amax per V channel (0 for an all-zero channel)
   float *mq, *dsk;
   long long *k_sum, *v_sum;      // fixed-point channel sums [B*Hkv][D]
   unsigned *v_max, *v_min;       // order-preserving keys of V channel max/min

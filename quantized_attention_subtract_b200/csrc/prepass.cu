@@ -6,10 +6,12 @@
 // ("SageAttention2: Technical report", section 2), Q and K are quantised per
 // block to INT8 and V to FP8 (closerAI ComfyUI blog, part 2).
 //
-// Three kernels on one stream:
+// Four kernels on one stream:
 //   kv_stats   per (b, kv head, 256-token chunk): fixed-point channel sums of
 //              K (and V) and the V channel max/min, combined with atomics
 //              (integer addition is exact, so the order does not matter);
+//   kv_finalize per (b, kv head): mean_k, mean_v, V channel scale and its
+//              reciprocal, once per channel;
 //   quantize   per 128-token tile of K, V or Q (in that order, K/V heads in
 //              reverse so their second read hits L2): smoothing, block amax,
 //              INT8/FP8 codes written through shared memory as whole
@@ -20,6 +22,7 @@
 //
 // Threads own 16-byte chunks (8 channels) of rows, so loads are 16-byte
 // vectors and a warp covers whole rows.
+#include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -31,8 +34,6 @@
 namespace sage {
 namespace {
 
-constexpr int kRowsPerPass = 16;   // rows handled concurrently by one CTA
-constexpr int kStatTokens = 256;   // tokens per kv_stats CTA
 constexpr float kTinyAmax = 0x1p-64f;  // blocks below this quantise to zero
 
 __device__ __forceinline__ void load8(const uint16_t *p, int bf16, float (&x)[8]) {
@@ -69,96 +70,221 @@ __device__ __forceinline__ long long fixed_point(float x) {
   return __float2ll_rn(__fmul_rn(x, kFixScale));
 }
 
+// ------------------------------------------------------------ streaming
+// Both streaming kernels are persistent: each block walks a list of units
+// (128-token tiles or 64-token chunks) and keeps the rows of the next units in
+// flight with cp.async.bulk copies into a ring of shared-memory stages, one
+// 16-byte-aligned row per copy (HND and NHD alike), completed on an mbarrier.
+constexpr int kStatChunk = 64;     // tokens per kv_stats unit
+
+__device__ __forceinline__ void decode8(uint4 u, int bf16, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint16_t lo = w[i] & 0xFFFFu, hi = w[i] >> 16;
+    if (bf16) {
+      x[2 * i] = __uint_as_float(uint32_t(lo) << 16);
+      x[2 * i + 1] = __uint_as_float(uint32_t(hi) << 16);
+    } else {
+      x[2 * i] = __half2float(__ushort_as_half(lo));
+      x[2 * i + 1] = __half2float(__ushort_as_half(hi));
+    }
+  }
+}
+
+// Issue the row copies of one unit: rows [0, nrows) of a tensor starting at
+// `src` with element stride `stride` between rows go to `dst` (row pitch
+// `rowb` bytes).  Called by every thread; thread t copies row t.  Thread 0
+// arms the barrier with the unit's byte count.
+__device__ __forceinline__ void issue_rows(uint32_t dst, const uint16_t *src, long long stride,
+                                           int nrows, int rowb, uint32_t bar, bool arm,
+                                           uint32_t total_bytes) {
+  if (arm && threadIdx.x == 0) mbar_arrive_expect_tx(bar, total_bytes);
+  if (int(threadIdx.x) < nrows) bulk_load(dst + threadIdx.x * rowb, src + threadIdx.x * stride, rowb, bar);
+}
+
+// Block-wide bounded wait; every thread learns whether it succeeded.
+__device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity, int *status) {
+  const bool ok = mbar_wait(bar, parity, status);
+  return __syncthreads_and(ok ? 1 : 0) != 0;
+}
+
 // ------------------------------------------------------------ kv_stats
-// grid (ceil(Nkv / 256), B * Hkv), block 16 * (D / 8).  Each thread owns one
-// 16-byte chunk (8 channels) and walks rows 16 apart, two rows per step so
-// that four 16-byte loads are in flight before any arithmetic.
+// Persistent, grid <= 2 per SM, block 256.  Units are 64-token chunks of one
+// (b, kv head), numbered bh * nchunks + chunk; block i takes a contiguous run
+// of units, so its partial sums stay in registers and are flushed (block
+// reduction + integer / ordered-key atomics) only when the head changes.
+// Stage: 64 K rows then 64 V rows (K only when smooth_k).
+constexpr int kStatStages = 2;
+
 __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace ws) {
-  const int C8 = pb.D / 8;
-  const int c8 = threadIdx.x % C8, r0 = threadIdx.x / C8;
-  const int bh = blockIdx.y, b = bh / pb.Hkv, h = bh % pb.Hkv;
-  const int j0 = blockIdx.x * kStatTokens;
-  const uint16_t *kb = pb.k + b * pb.ks_b + h * pb.ks_h + 8 * c8;
-  const uint16_t *vb = pb.v + b * pb.vs_b + h * pb.vs_h + 8 * c8;
+  extern __shared__ __align__(128) uint8_t sm_stats[];
+  const int D = pb.D, C8 = D / 8, rowb = 2 * D;
+  const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;   // 16 / 21 / 32 row groups
+  const int ngroups = blockDim.x / C8;
+  const int nchunk = (pb.Nkv + kStatChunk - 1) / kStatChunk;
+  const long long nunits = (long long)pb.B * pb.Hkv * nchunk;
+  const long long u0 = nunits * blockIdx.x / gridDim.x, u1 = nunits * (blockIdx.x + 1) / gridDim.x;
+  const int stage_bytes = 2 * kStatChunk * rowb;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm_stats + kStatStages * stage_bytes);
+  long long *red = reinterpret_cast<long long *>(bars + 8);         // [ngroups][D]
+  const uint32_t s_base = smem_u32(sm_stats), b_base = smem_u32(bars);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStatStages; ++i) mbar_init(b_base + 8 * i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  auto unit_src = [&](long long u, int &bh, int &j0, int &n) {
+    bh = int(u / nchunk);
+    j0 = int(u % nchunk) * kStatChunk;
+    n = min(kStatChunk, pb.Nkv - j0);
+  };
+  auto issue = [&](long long u, int st) {
+    int bh, j0, n;
+    unit_src(u, bh, j0, n);
+    const int b = bh / pb.Hkv, h = bh % pb.Hkv;
+    const uint32_t dst = s_base + st * stage_bytes, bar = b_base + 8 * st;
+    const uint32_t bytes = uint32_t(n) * rowb * (pb.smooth_k ? 2 : 1);
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, bytes);
+    if (pb.smooth_k && int(threadIdx.x) < n)
+      bulk_load(dst + threadIdx.x * rowb, pb.k + b * pb.ks_b + h * pb.ks_h + (j0 + threadIdx.x) * pb.ks_n,
+                rowb, bar);
+    if (int(threadIdx.x) >= 128 - n && threadIdx.x < 128) {
+      const int r = threadIdx.x - (128 - n);
+      bulk_load(dst + (kStatChunk + r) * rowb,
+                pb.v + b * pb.vs_b + h * pb.vs_h + (j0 + r) * pb.vs_n, rowb, bar);
+    }
+  };
 
   long long ksum[8], vsum[8];
   float vmax[8], vmin[8];
+  auto reset = [&]() {
 #pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    ksum[e] = 0;
-    vsum[e] = 0;
-    vmax[e] = -INFINITY;
-    vmin[e] = INFINITY;
-  }
-  for (int rr = r0; rr < kStatTokens; rr += 2 * kRowsPerPass) {
-    float xk[2][8], xv[2][8];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = j0 + rr + u * kRowsPerPass;
-      if (j < pb.Nkv) {
-        if (pb.smooth_k) load8(kb + j * pb.ks_n, pb.bf16, xk[u]);
-        load8(vb + j * pb.vs_n, pb.bf16, xv[u]);
-      }
+    for (int e = 0; e < 8; ++e) {
+      ksum[e] = 0;
+      vsum[e] = 0;
+      vmax[e] = -INFINITY;
+      vmin[e] = INFINITY;
     }
+  };
+  auto flush = [&](int bh) {
+    const bool live = rg < ngroups;
+    if (pb.smooth_k) {
+      if (live)
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = j0 + rr + u * kRowsPerPass;
-      if (j < pb.Nkv) {
+        for (int e = 0; e < 8; ++e) red[rg * D + 8 * c8 + e] = ksum[e];
+      __syncthreads();
+      if (int(threadIdx.x) < D) {
+        long long t = 0;
+        for (int r = 0; r < ngroups; ++r) t += red[r * D + threadIdx.x];
+        atomicAdd(reinterpret_cast<unsigned long long *>(ws.k_sum + (long long)bh * D + threadIdx.x),
+                  (unsigned long long)t);
+      }
+      __syncthreads();
+    }
+    if (pb.smooth_v) {
+      if (live)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[rg * D + 8 * c8 + e] = vsum[e];
+      __syncthreads();
+      if (int(threadIdx.x) < D) {
+        long long t = 0;
+        for (int r = 0; r < ngroups; ++r) t += red[r * D + threadIdx.x];
+        atomicAdd(reinterpret_cast<unsigned long long *>(ws.v_sum + (long long)bh * D + threadIdx.x),
+                  (unsigned long long)t);
+      }
+      __syncthreads();
+    }
+    float *redf = reinterpret_cast<float *>(red);
+    if (live)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        redf[rg * D + 8 * c8 + e] = vmax[e];
+        redf[(ngroups + rg) * D + 8 * c8 + e] = vmin[e];
+      }
+    __syncthreads();
+    if (int(threadIdx.x) < D) {
+      float mx = -INFINITY, mn = INFINITY;
+      for (int r = 0; r < ngroups; ++r) {
+        mx = fmaxf(mx, redf[r * D + threadIdx.x]);
+        mn = fminf(mn, redf[(ngroups + r) * D + threadIdx.x]);
+      }
+      atomicMax(ws.v_max + (long long)bh * D + threadIdx.x, float_key(mx));
+      atomicMin(ws.v_min + (long long)bh * D + threadIdx.x, float_key(mn));
+    }
+    __syncthreads();
+  };
+
+  reset();
+  for (int i = 0; i < kStatStages; ++i)
+    if (u0 + i < u1) issue(u0 + i, i);
+  int cur_bh = -1;
+  bool ok = true;
+  for (long long u = u0; u < u1; ++u) {
+    const int it = int(u - u0), st = it % kStatStages;
+    if (!block_wait(b_base + 8 * st, (it / kStatStages) & 1, ws.status)) { ok = false; break; }
+    int bh, j0, n;
+    unit_src(u, bh, j0, n);
+    if (bh != cur_bh) {
+      if (cur_bh >= 0) flush(cur_bh);
+      reset();
+      cur_bh = bh;
+    }
+    const uint8_t *stage = sm_stats + st * stage_bytes;
+    if (rg < ngroups) {
+      for (int r = rg; r < n; r += ngroups) {
+        float x[8];
+        if (pb.smooth_k) {
+          decode8(*reinterpret_cast<const uint4 *>(stage + r * rowb + 16 * c8), pb.bf16, x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ksum[e] += fixed_point(x[e]);
+        }
+        decode8(*reinterpret_cast<const uint4 *>(stage + (kStatChunk + r) * rowb + 16 * c8), pb.bf16, x);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          if (pb.smooth_k) ksum[e] += fixed_point(xk[u][e]);
-          vmax[e] = fmaxf(vmax[e], xv[u][e]);
-          vmin[e] = fminf(vmin[e], xv[u][e]);
-          if (pb.smooth_v) vsum[e] += fixed_point(xv[u][e]);
+          vmax[e] = fmaxf(vmax[e], x[e]);
+          vmin[e] = fminf(vmin[e], x[e]);
+          if (pb.smooth_v) vsum[e] += fixed_point(x[e]);
         }
       }
     }
+    __syncthreads();  // stage consumed
+    if (u + kStatStages < u1) issue(u + kStatStages, st);
   }
+  if (ok && cur_bh >= 0) flush(cur_bh);
+  if (!ok) {
+    // wait (bounded) for every copy still in flight before leaving
+    for (long long u = u0; u < u1 && u < u0 + kStatStages; ++u) {
+      const int it = int(u - u0);
+      mbar_wait(b_base + 8 * (it % kStatStages), (it / kStatStages) & 1, ws.status, false);
+    }
+  }
+}
 
-  // Combine the 16 row groups per channel through shared memory.
-  __shared__ long long red[kRowsPerPass][128];
-  const int D = pb.D;
-  const int tid = threadIdx.x;
-  long long *ks_out = ws.k_sum + (long long)bh * D;
-  long long *vs_out = ws.v_sum + (long long)bh * D;
-  if (pb.smooth_k) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[r0][8 * c8 + e] = ksum[e];
-    __syncthreads();
-    if (tid < D) {
-      long long s = 0;
-      for (int r = 0; r < kRowsPerPass; ++r) s += red[r][tid];
-      atomicAdd(reinterpret_cast<unsigned long long *>(ks_out + tid), (unsigned long long)s);
-    }
-    __syncthreads();
+// ------------------------------------------------------------ kv_finalize
+// grid B * Hkv, block D: the per-channel constants every K and V tile of a
+// head uses, computed once: mean_k (exact fixed-point mean), mean_v, and the
+// V channel scale amax/448 with its reciprocal 448/amax (IEEE fp32 division;
+// amax = max |fl(v - mean_v)| taken from the channel max and min, which is
+// exact because fl(v - mean) is monotone in v).
+__global__ void kv_finalize_kernel(Problem pb, Workspace ws) {
+  const int c = threadIdx.x;
+  const long long ci = (long long)blockIdx.x * pb.D + c;
+  if (c >= pb.D) return;
+  ws.mean_k[ci] = pb.smooth_k ? fixed_mean(ws.k_sum[ci], pb.Nkv) : 0.f;
+  const float mv = pb.smooth_v ? fixed_mean(ws.v_sum[ci], pb.Nkv) : 0.f;
+  ws.mean_v[ci] = mv;
+  const float hi = __fsub_rn(key_float(ws.v_max[ci]), mv);
+  const float lo = __fsub_rn(key_float(ws.v_min[ci]), mv);
+  const float a = fmaxf(fabsf(hi), fabsf(lo));
+  float sc = 0.f, inv = 0.f;
+  if (a >= kTinyAmax) {
+    sc = __fdiv_rn(a, 448.0f);
+    inv = __fdiv_rn(448.0f, a);
   }
-  if (pb.smooth_v) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[r0][8 * c8 + e] = vsum[e];
-    __syncthreads();
-    if (tid < D) {
-      long long s = 0;
-      for (int r = 0; r < kRowsPerPass; ++r) s += red[r][tid];
-      atomicAdd(reinterpret_cast<unsigned long long *>(vs_out + tid), (unsigned long long)s);
-    }
-    __syncthreads();
-  }
-  float *redf = reinterpret_cast<float *>(&red[0][0]);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    redf[r0 * 128 + 8 * c8 + e] = vmax[e];
-    redf[kRowsPerPass * 128 + r0 * 128 + 8 * c8 + e] = vmin[e];
-  }
-  __syncthreads();
-  if (tid < D) {
-    float mx = -INFINITY, mn = INFINITY;
-    for (int r = 0; r < kRowsPerPass; ++r) {
-      mx = fmaxf(mx, redf[r * 128 + tid]);
-      mn = fminf(mn, redf[kRowsPerPass * 128 + r * 128 + tid]);
-    }
-    atomicMax(ws.v_max + (long long)bh * D + tid, float_key(mx));
-    atomicMin(ws.v_min + (long long)bh * D + tid, float_key(mn));
-  }
+  ws.v_scale[ci] = sc;
+  ws.v_inv[ci] = inv;
 }
 
 // Block-wide max of two values (one per K half, or the same value twice);
@@ -184,10 +310,16 @@ __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
   }
 }
 
-__device__ __forceinline__ uint32_t int8_code(float x, float inv) {
-  int q = __float2int_rn(__fmul_rn(x, inv));
-  q = q > 127 ? 127 : (q < -127 ? -127 : q);
-  return uint32_t(q) & 0xFFu;
+// INT8 code of x with reciprocal scale inv: rint(fl(x * inv)), round half to
+// even.  Adding 1.5 * 2^23 in fp32 rounds to an integer exactly that way and
+// leaves it (two's complement) in the low mantissa bits; |fl(x * inv)| is at
+// most 127 * (1 + 2^-24), so the code is always in [-127, 127].
+__device__ __forceinline__ uint32_t int8_bits(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
+}
+// Pack the low bytes of four such words (first in bits [0, 8)).
+__device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Copy a finished [rows][row_bytes] tile from shared memory to a contiguous
@@ -198,58 +330,120 @@ __device__ __forceinline__ void store_tile(uint8_t *dst, const uint8_t *src, int
 }
 
 // ------------------------------------------------------------ quantize
-// grid (nK + nV + nQ), block 32 * (D / 8): thread t owns channels
+// Persistent, grid <= 2 per SM, block 32 * (D / 8): thread t owns channels
 // 8 * (t % (D/8)) .. +7 of the four consecutive rows 4 * (t / (D/8)) .. +3 of
-// one 128-token tile.  Block order: K and V tiles first, heads in reverse
-// order (those kv_stats read last are still in L2), then Q blocks.
-__global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws) {
-  __shared__ __align__(16) uint8_t tile[128 * 128];
-  __shared__ unsigned long long colsum[128];
-  __shared__ float chan[128];
-  __shared__ float scratch[64];
+// a 128-token tile.  Units: K and V tiles first, heads in reverse order
+// (those kv_stats read last may still be in L2), then Q blocks; block i takes
+// units i, i + grid, ...  Two input stages of 128 rows are kept in flight.
+constexpr int kQuantStages = 2;
 
-  const int D = pb.D, Dp = ws.Dp, C8 = D / 8;
-  const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;  // rows 4 rg .. 4 rg + 3
+struct QUnit {
+  int kind;  // 0 = K tile, 1 = V tile, 2 = Q block
+  int bh, t, b, h, r0, nvalid;
+  const uint16_t *src;
+  long long stride;
+};
+
+__device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &ws, long long u) {
+  QUnit q{};
   const int nKt = ws.Nkv_pad / kKVTile;
-  const int nKV = pb.B * pb.Hkv * nKt;
-  int blk = blockIdx.x;
-  float x[4][8];
+  const long long nKV = (long long)pb.B * pb.Hkv * nKt;
+  if (u < 2 * nKV) {
+    q.kind = int(u & 1);
+    const long long kvi = nKV - 1 - (u >> 1);  // reverse head order
+    q.t = int(kvi % nKt);
+    q.bh = int(kvi / nKt);
+    q.b = q.bh / pb.Hkv;
+    q.h = q.bh % pb.Hkv;
+    q.r0 = q.t * kKVTile;
+    q.nvalid = max(0, min(kKVTile, pb.Nkv - q.r0));
+    if (q.kind == 0) {
+      q.src = pb.k + q.b * pb.ks_b + q.h * pb.ks_h + q.r0 * pb.ks_n;
+      q.stride = pb.ks_n;
+    } else {
+      q.src = pb.v + q.b * pb.vs_b + q.h * pb.vs_h + q.r0 * pb.vs_n;
+      q.stride = pb.vs_n;
+    }
+  } else {
+    const long long qi = u - 2 * nKV;
+    q.kind = 2;
+    q.t = int(qi % ws.nqb);
+    q.bh = int(qi / ws.nqb);
+    q.b = q.bh / pb.Hq;
+    q.h = q.bh % pb.Hq;
+    q.r0 = q.t * kQBlk;
+    q.nvalid = min(kQBlk, pb.Nq - q.r0);
+    q.src = pb.q + q.b * pb.qs_b + q.h * pb.qs_h + q.r0 * pb.qs_n;
+    q.stride = pb.qs_n;
+  }
+  return q;
+}
 
-  if (blk < 2 * nKV) {
-    const int isV = blk & 1;
-    const int kvi = nKV - 1 - (blk >> 1);  // reverse head order
-    const int kt = kvi % nKt, bh = kvi / nKt, b = bh / pb.Hkv, h = bh % pb.Hkv;
-    const int j0 = kt * kKVTile, nvalid = max(0, min(kKVTile, pb.Nkv - j0));
-    if (!isV) {
+__global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws) {
+  extern __shared__ __align__(128) uint8_t sm_q[];
+  const int D = pb.D, Dp = ws.Dp, C8 = D / 8, rowb = 2 * D;
+  const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;  // rows 4 rg .. 4 rg + 3
+  const int stage_bytes = 128 * rowb;
+  uint8_t *tile = sm_q + kQuantStages * stage_bytes;        // output codes [128][128]
+  uint64_t *bars = reinterpret_cast<uint64_t *>(tile + 128 * 128);
+  unsigned long long *colsum = reinterpret_cast<unsigned long long *>(bars + 4);
+  float *chan = reinterpret_cast<float *>(colsum + 128);
+  float *scratch = chan + 128;
+  const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
+  const int nKt = ws.Nkv_pad / kKVTile;
+  const long long nunits = 2LL * pb.B * pb.Hkv * nKt + (long long)pb.B * pb.Hq * ws.nqb;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kQuantStages; ++i) mbar_init(b_base + 8 * i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  auto issue = [&](long long u, int st) {
+    const QUnit q = quant_unit(pb, ws, u);
+    issue_rows(s_base + st * stage_bytes, q.src, q.stride, q.nvalid, rowb, b_base + 8 * st, true,
+               uint32_t(q.nvalid) * rowb);
+  };
+  for (int i = 0; i < kQuantStages; ++i)
+    if (blockIdx.x + (long long)i * gridDim.x < nunits) issue(blockIdx.x + (long long)i * gridDim.x, i);
+
+  float x[4][8];
+  int it = 0;
+  bool ok = true;
+  for (long long u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+    const int st = it % kQuantStages;
+    if (!block_wait(b_base + 8 * st, (it / kQuantStages) & 1, ws.status)) { ok = false; break; }
+    const QUnit q = quant_unit(pb, ws, u);
+    const uint8_t *stage = sm_q + st * stage_bytes;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = 4 * rg + r;
+      if (row < q.nvalid) decode8(*reinterpret_cast<const uint4 *>(stage + row * rowb + 16 * c8), pb.bf16, x[r]);
+      else
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
+    }
+    __syncthreads();  // stage consumed: refill it with the unit after next
+    const long long un = u + (long long)kQuantStages * gridDim.x;
+    if (un < nunits) issue(un, st);
+
+    if (q.kind == 0) {
       // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
-      const uint16_t *src = pb.k + b * pb.ks_b + h * pb.ks_h + 8 * c8;
       float mean[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        mean[e] = pb.smooth_k ? fixed_mean(ws.k_sum[(long long)bh * D + 8 * c8 + e], pb.Nkv) : 0.f;
-      if (kt == 0 && rg == 0)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ws.mean_k[(long long)bh * D + 8 * c8 + e] = mean[e];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = 4 * rg + u;
-        if (r < nvalid) load8(src + (long long)(j0 + r) * pb.ks_n, pb.bf16, x[u]);
+      {
+        const float4 *mk = reinterpret_cast<const float4 *>(ws.mean_k + (long long)q.bh * D + 8 * c8);
+        const float4 m0 = __ldg(mk), m1 = __ldg(mk + 1);
+        mean[0] = m0.x; mean[1] = m0.y; mean[2] = m0.z; mean[3] = m0.w;
+        mean[4] = m1.x; mean[5] = m1.y; mean[6] = m1.z; mean[7] = m1.w;
       }
       float a = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (4 * rg + u < nvalid) {
+      for (int r = 0; r < 4; ++r)
+        if (4 * rg + r < q.nvalid)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            x[u][e] = __fsub_rn(x[u][e], mean[e]);
-            a = fmaxf(a, fabsf(x[u][e]));
+            x[r][e] = __fsub_rn(x[r][e], mean[e]);
+            a = fmaxf(a, fabsf(x[r][e]));
           }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
-        }
-      }
-      // rows 0..63 belong to block 2 kt, rows 64..127 to 2 kt + 1
+      // rows 0..63 belong to block 2 t, rows 64..127 to 2 t + 1
       float a0 = rg < 16 ? a : 0.f, a1 = rg < 16 ? 0.f : a;
       block_max2(a0, a1, scratch);
       float inv0 = 0.f, inv1 = 0.f, s0 = 0.f, s1 = 0.f;
@@ -262,8 +456,8 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
         inv1 = __fdiv_rn(127.0f, a1);
       }
       if (threadIdx.x == 0) {
-        ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt] = s0;
-        ws.k_scale[(long long)bh * (ws.Nkv_pad / kKBlk) + 2 * kt + 1] = s1;
+        ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 2 * q.t] = s0;
+        ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 2 * q.t + 1] = s1;
       }
       const float inv = rg < 16 ? inv0 : inv1;
       if (Dp != D)
@@ -271,152 +465,127 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
           *reinterpret_cast<uint32_t *>(tile + o) = 0u;
       __syncthreads();
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          w0 |= int8_code(x[u][e], inv) << (8 * e);
-          w1 |= int8_code(x[u][e + 4], inv) << (8 * e);
-        }
-        *reinterpret_cast<uint2 *>(tile + (4 * rg + u) * Dp + 8 * c8) = make_uint2(w0, w1);
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
+                                     int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
+        const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
+                                     int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
+        *reinterpret_cast<uint2 *>(tile + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
       }
       __syncthreads();
-      store_tile(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)bh * ws.Nkv_pad + j0) * Dp, tile,
+      store_tile(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, tile,
                  128 * Dp);
-      return;
-    }
-    // ---------------- V tile: V' = V - mean_v, FP8 per channel, transposed
-    const uint16_t *src = pb.v + b * pb.vs_b + h * pb.vs_h + 8 * c8;
-    float mean[8], inv[8];
+    } else if (q.kind == 1) {
+      // ---------------- V tile: V' = V - mean_v, FP8 per channel, transposed
+      float mean[8], inv[8];
+      {
+        const float4 *mv = reinterpret_cast<const float4 *>(ws.mean_v + (long long)q.bh * D + 8 * c8);
+        const float4 *iv = reinterpret_cast<const float4 *>(ws.v_inv + (long long)q.bh * D + 8 * c8);
+        const float4 m0 = __ldg(mv), m1 = __ldg(mv + 1), i0 = __ldg(iv), i1 = __ldg(iv + 1);
+        mean[0] = m0.x; mean[1] = m0.y; mean[2] = m0.z; mean[3] = m0.w;
+        mean[4] = m1.x; mean[5] = m1.y; mean[6] = m1.z; mean[7] = m1.w;
+        inv[0] = i0.x; inv[1] = i0.y; inv[2] = i0.z; inv[3] = i0.w;
+        inv[4] = i1.x; inv[5] = i1.y; inv[6] = i1.z; inv[7] = i1.w;
+      }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const long long ci = (long long)bh * D + 8 * c8 + e;
-      mean[e] = pb.smooth_v ? fixed_mean(ws.v_sum[ci], pb.Nkv) : 0.f;
-      const float hi = __fsub_rn(key_float(ws.v_max[ci]), mean[e]);
-      const float lo = __fsub_rn(key_float(ws.v_min[ci]), mean[e]);
-      const float a = fmaxf(fabsf(hi), fabsf(lo));
-      float sc = 0.f;
-      inv[e] = 0.f;
+      for (int r = 0; r < 4; ++r) {
+        if (4 * rg + r < q.nvalid) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[r][e] = __fmul_rn(__fsub_rn(x[r][e], mean[e]), inv[e]);
+        }
+      }
+      // Transposed tile [D][128 keys] as 32 words per channel row; the word of
+      // keys 4 rg .. 4 rg + 3 of channel c sits at position (rg + rot * c8) % 32,
+      // which puts the 32 lanes of a warp on 32 different banks.
+      const int rot = 32 / (C8 == 12 ? 16 : C8);
+      uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
+#pragma unroll
+      for (int e = 0; e < 8; e += 2) {
+        uint32_t w_lo = 0, w_hi = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const uint32_t pr = e4m3x2(x[r][e], x[r][e + 1]);
+          w_lo |= (pr & 0xFFu) << (8 * r);
+          w_hi |= (pr >> 8) << (8 * r);
+        }
+        const int pos = (rg + rot * c8) & 31;
+        tw[(8 * c8 + e) * 32 + pos] = w_lo;
+        tw[(8 * c8 + e + 1) * 32 + pos] = w_hi;
+      }
+      __syncthreads();
+      uint8_t *dst = ws.v8t + (long long)q.bh * D * ws.Nkv_pad + q.r0;
+      for (int t = threadIdx.x; t < D * 8; t += blockDim.x) {
+        const int c = t >> 3, qq = t & 7;  // channel row c, keys 16 qq .. 16 qq + 15
+        const int sh = rot * (c >> 3);
+        uint4 o;
+        o.x = tw[c * 32 + ((4 * qq + 0 + sh) & 31)];
+        o.y = tw[c * 32 + ((4 * qq + 1 + sh) & 31)];
+        o.z = tw[c * 32 + ((4 * qq + 2 + sh) & 31)];
+        o.w = tw[c * 32 + ((4 * qq + 3 + sh) & 31)];
+        *reinterpret_cast<uint4 *>(dst + (long long)c * ws.Nkv_pad + 16 * qq) = o;
+      }
+    } else {
+      // ---------------- Q block: optional block mean, INT8 per block
+      if (pb.smooth_q) {
+        if (int(threadIdx.x) < D) colsum[threadIdx.x] = 0ull;
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          long long s = 0;
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            if (4 * rg + r < q.nvalid) s += fixed_point(x[r][e]);
+          atomicAdd(&colsum[8 * c8 + e], (unsigned long long)s);
+        }
+        __syncthreads();
+        if (int(threadIdx.x) < D) {
+          const float m = fixed_mean((long long)colsum[threadIdx.x], q.nvalid);
+          chan[threadIdx.x] = m;
+          ws.mq[((long long)q.bh * ws.nqb + q.t) * D + threadIdx.x] = m;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+          if (4 * rg + r < q.nvalid)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], chan[8 * c8 + e]);
+      }
+      float a = 0.f, unused = 0.f;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[r][e]));
+      block_max2(a, unused, scratch);
+      float inv = 0.f, scale = 0.f;
       if (a >= kTinyAmax) {
-        sc = __fdiv_rn(a, 448.0f);
-        inv[e] = __fdiv_rn(448.0f, a);
+        scale = __fdiv_rn(a, 127.0f);
+        inv = __fdiv_rn(127.0f, a);
       }
-      if (kt == 0 && rg == 0) {
-        ws.v_scale[ci] = sc;
-        ws.mean_v[ci] = mean[e];
+      if (threadIdx.x == 0) ws.q_scale[(long long)q.bh * ws.nqb + q.t] = scale;
+      if (Dp != D)
+        for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
+          *reinterpret_cast<uint32_t *>(tile + o) = 0u;
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
+                                     int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
+        const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
+                                     int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
+        *reinterpret_cast<uint2 *>(tile + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
       }
+      __syncthreads();
+      store_tile(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, tile,
+                 128 * Dp);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = 4 * rg + u;
-      if (r < nvalid) {
-        load8(src + (long long)(j0 + r) * pb.vs_n, pb.bf16, x[u]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[u][e] = __fmul_rn(__fsub_rn(x[u][e], mean[e]), inv[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
-      }
-    }
-    // Transposed tile [D][128 keys] as 32 words per channel row; the word of
-    // keys 4 rg .. 4 rg + 3 of channel c sits at position (rg + rot * c8) % 32,
-    // which puts the 32 lanes of a warp on 32 different banks.
-    const int rot = 32 / (C8 == 12 ? 16 : C8);
-    uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      uint32_t w_lo = 0, w_hi = 0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t pr = e4m3x2(x[u][e], x[u][e + 1]);
-        w_lo |= (pr & 0xFFu) << (8 * u);
-        w_hi |= (pr >> 8) << (8 * u);
-      }
-      const int pos = (rg + rot * c8) & 31;
-      tw[(8 * c8 + e) * 32 + pos] = w_lo;
-      tw[(8 * c8 + e + 1) * 32 + pos] = w_hi;
-    }
-    __syncthreads();
-    uint8_t *dst = ws.v8t + (long long)bh * D * ws.Nkv_pad + j0;
-    for (int t = threadIdx.x; t < D * 8; t += blockDim.x) {
-      const int c = t >> 3, q = t & 7;  // channel row c, keys 16 q .. 16 q + 15
-      const int sh = rot * (c >> 3);
-      uint4 o;
-      o.x = tw[c * 32 + ((4 * q + 0 + sh) & 31)];
-      o.y = tw[c * 32 + ((4 * q + 1 + sh) & 31)];
-      o.z = tw[c * 32 + ((4 * q + 2 + sh) & 31)];
-      o.w = tw[c * 32 + ((4 * q + 3 + sh) & 31)];
-      *reinterpret_cast<uint4 *>(dst + (long long)c * ws.Nkv_pad + 16 * q) = o;
-    }
-    return;
+    __syncthreads();  // output tile free for the next unit
   }
-  blk -= 2 * nKV;
-  {
-    // ---------------- Q block: optional block mean, INT8 per block
-    const int qb = blk % ws.nqb, bh = blk / ws.nqb, b = bh / pb.Hq, h = bh % pb.Hq;
-    const int i0 = qb * kQBlk, nvalid = min(kQBlk, pb.Nq - i0);
-    const uint16_t *src = pb.q + b * pb.qs_b + h * pb.qs_h + 8 * c8;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = 4 * rg + u;
-      if (r < nvalid) load8(src + (long long)(i0 + r) * pb.qs_n, pb.bf16, x[u]);
-      else
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[u][e] = 0.f;
+  if (!ok) {
+    // wait (bounded) for copies still in flight before leaving
+    for (int i = 0; i < kQuantStages; ++i) {
+      const long long u = blockIdx.x + (long long)(it + i) * gridDim.x;
+      if (u < nunits) mbar_wait(b_base + 8 * ((it + i) % kQuantStages), ((it + i) / kQuantStages) & 1, ws.status, false);
     }
-    if (pb.smooth_q) {
-      if (threadIdx.x < D) colsum[threadIdx.x] = 0ull;
-      __syncthreads();
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        long long s = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (4 * rg + u < nvalid) s += fixed_point(x[u][e]);
-        atomicAdd(&colsum[8 * c8 + e], (unsigned long long)s);
-      }
-      __syncthreads();
-      if (threadIdx.x < D) {
-        const float m = fixed_mean((long long)colsum[threadIdx.x], nvalid);
-        chan[threadIdx.x] = m;
-        ws.mq[((long long)bh * ws.nqb + qb) * D + threadIdx.x] = m;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (4 * rg + u < nvalid)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[u][e] = __fsub_rn(x[u][e], chan[8 * c8 + e]);
-    }
-    float a = 0.f, unused = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[u][e]));
-    block_max2(a, unused, scratch);
-    float inv = 0.f, scale = 0.f;
-    if (a >= kTinyAmax) {
-      scale = __fdiv_rn(a, 127.0f);
-      inv = __fdiv_rn(127.0f, a);
-    }
-    if (threadIdx.x == 0) ws.q_scale[(long long)bh * ws.nqb + qb] = scale;
-    if (Dp != D)
-      for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
-        *reinterpret_cast<uint32_t *>(tile + o) = 0u;
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      uint32_t w0 = 0, w1 = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        w0 |= int8_code(x[u][e], inv) << (8 * e);
-        w1 |= int8_code(x[u][e + 4], inv) << (8 * e);
-      }
-      *reinterpret_cast<uint2 *>(tile + (4 * rg + u) * Dp + 8 * c8) = make_uint2(w0, w1);
-    }
-    __syncthreads();
-    store_tile(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)bh * ws.Nq_pad + i0) * Dp, tile,
-               128 * Dp);
   }
 }
 
@@ -473,13 +642,32 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(ws.v_min, 0xFF, nch * sizeof(unsigned), stream);
   if (e != cudaSuccess) return e;
-  dim3 g1((pb.Nkv + kStatTokens - 1) / kStatTokens, pb.B * pb.Hkv);
-  kv_stats_kernel<<<g1, 16 * (pb.D / 8), 0, stream>>>(pb, ws);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // kv_stats: persistent, 2 blocks per SM
+  const int rowb = 2 * pb.D;
+  const int ngroups = 256 / (pb.D / 8);
+  const size_t st_smem = kStatStages * 2 * kStatChunk * rowb + 64 + sizeof(long long) * ngroups * pb.D;
+  e = cudaFuncSetAttribute(kv_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)st_smem);
+  if (e != cudaSuccess) return e;
+  const long long nchunk = (pb.Nkv + kStatChunk - 1) / kStatChunk;
+  const long long su = (long long)pb.B * pb.Hkv * nchunk;
+  const unsigned g1 = (unsigned)std::min<long long>(su, 2LL * sms);
+  kv_stats_kernel<<<g1, 256, st_smem, stream>>>(pb, ws);
   e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  kv_finalize_kernel<<<pb.B * pb.Hkv, 128, 0, stream>>>(pb, ws);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // quantize: persistent, 2 blocks per SM
+  const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 64 * 4;
+  e = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
   if (e != cudaSuccess) return e;
   const int nKt = ws.Nkv_pad / kKVTile;
   const long long nblk = (long long)pb.B * pb.Hq * ws.nqb + 2LL * pb.B * pb.Hkv * nKt;
-  quantize_kernel<<<dim3((unsigned)nblk), 32 * (pb.D / 8), 0, stream>>>(pb, ws);
+  const unsigned g2 = (unsigned)std::min<long long>(nblk, 2LL * sms);
+  quantize_kernel<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (pb.smooth_q) {

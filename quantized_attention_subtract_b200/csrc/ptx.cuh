@@ -95,6 +95,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
       : "memory");
 }
 
+// Contiguous bulk copy global -> shared (no tensor map), completion counted
+// in bytes on `bar`.  Both addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy
 // (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -261,6 +271,26 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Exact int32 -> fp32 for |s| < 2^22 (|S| <= 127^2 * 128 < 2^21 here) on the
+// integer and FMA pipes: the bits 0x4B400000 + s are the float 1.5 * 2^23 + s,
+// and subtracting 1.5 * 2^23 is exact.
+__device__ __forceinline__ float s32_to_f32_exact(uint32_t s) {
+  return __fsub_rn(__uint_as_float(s + 0x4B400000u), 12582912.0f);
+}
+
+// Four fp32 -> four FP8 e4m3 codes packed in one word, a in bits [0,8), b in
+// [8,16), c in [16,24), d in [24,32) (round to nearest even, saturating).
+__device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
+  uint32_t w;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(w)
+      : "f"(a), "f"(b), "f"(c), "f"(d));
+  return w;
 }
 
 // Two fp32 -> two FP8 e4m3 codes (round to nearest even, saturating to

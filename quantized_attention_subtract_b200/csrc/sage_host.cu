@@ -27,7 +27,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t off_q8, off_k8, off_v8t, off_qs, off_ks, off_vs, off_mk, off_mv, off_mq, off_dsk;
-  size_t off_ksum, off_vsum, off_vmax, off_vmin, off_status, total;
+  size_t off_ksum, off_vsum, off_vmax, off_vmin, off_vinv, off_status, total;
   int Dp, Nq_pad, Nkv_pad, nqb, nkb;
 };
 
@@ -84,6 +84,7 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.off_vmax = o;
   o = align_up(o + BHk * D * sizeof(unsigned), kAlign);
   L.off_vmin = take(BHk * D * sizeof(unsigned));
+  L.off_vinv = take(BHk * D * sizeof(float));
   L.off_status = take(16);
   if (p->smooth_q) {
     L.off_mq = take(BHq * L.nqb * D * sizeof(float));
@@ -112,6 +113,7 @@ Workspace make_workspace(const sage_attn_params_t *p, const Layout &L) {
   ws.v_sum = reinterpret_cast<long long *>(w + L.off_vsum);
   ws.v_max = reinterpret_cast<unsigned *>(w + L.off_vmax);
   ws.v_min = reinterpret_cast<unsigned *>(w + L.off_vmin);
+  ws.v_inv = reinterpret_cast<float *>(w + L.off_vinv);
   ws.status = reinterpret_cast<int *>(w + L.off_status);
   ws.Dp = L.Dp;
   ws.Nq_pad = L.Nq_pad;
