@@ -288,7 +288,8 @@ __global__ void kv_finalize_kernel(Problem pb, Workspace ws) {
 }
 
 // Block-wide max of two values (one per K half, or the same value twice);
-// up to 32 warps.
+// up to 32 warps.  Warp partials meet in shared memory, warp 0 reduces them
+// and broadcasts the result.
 __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -296,18 +297,26 @@ __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
     b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
   }
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
-  __syncthreads();
   if (lane == 0) {
     scratch[warp] = a;
     scratch[32 + warp] = b;
   }
   __syncthreads();
-  a = scratch[0];
-  b = scratch[32];
-  for (int w = 1; w < nw; ++w) {
-    a = fmaxf(a, scratch[w]);
-    b = fmaxf(b, scratch[32 + w]);
+  if (warp == 0) {
+    float x = lane < nw ? scratch[lane] : 0.f, y = lane < nw ? scratch[32 + lane] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+      y = fmaxf(y, __shfl_xor_sync(0xffffffffu, y, o));
+    }
+    if (lane == 0) {
+      scratch[64] = x;
+      scratch[65] = y;
+    }
   }
+  __syncthreads();
+  a = scratch[64];
+  b = scratch[65];
 }
 
 // INT8 code of x with reciprocal scale inv: rint(fl(x * inv)), round half to
@@ -388,7 +397,8 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   uint64_t *bars = reinterpret_cast<uint64_t *>(tile + 128 * 128);
   unsigned long long *colsum = reinterpret_cast<unsigned long long *>(bars + 4);
   float *chan = reinterpret_cast<float *>(colsum + 128);
-  float *scratch = chan + 128;
+  float *scratch = chan + 128;                               // 66 floats
+  QUnit *desc = reinterpret_cast<QUnit *>(scratch + 72);    // [stages + 1]
   const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
   const int nKt = ws.Nkv_pad / kKVTile;
   const long long nunits = 2LL * pb.B * pb.Hkv * nKt + (long long)pb.B * pb.Hq * ws.nqb;
@@ -397,13 +407,20 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
     fence_mbar_init();
   }
   __syncthreads();
-  auto issue = [&](long long u, int st) {
-    const QUnit q = quant_unit(pb, ws, u);
+  // Unit descriptors are decoded once, by thread 0, into shared memory:
+  // desc[st] describes the unit whose rows are in (or on their way into)
+  // stage st; desc[kQuantStages] is the next one to issue.
+  auto issue = [&](const QUnit &q, int st) {
     issue_rows(s_base + st * stage_bytes, q.src, q.stride, q.nvalid, rowb, b_base + 8 * st, true,
                uint32_t(q.nvalid) * rowb);
   };
+  if (threadIdx.x == 0)
+    for (int i = 0; i < kQuantStages; ++i)
+      if (blockIdx.x + (long long)i * gridDim.x < nunits)
+        desc[i] = quant_unit(pb, ws, blockIdx.x + (long long)i * gridDim.x);
+  __syncthreads();
   for (int i = 0; i < kQuantStages; ++i)
-    if (blockIdx.x + (long long)i * gridDim.x < nunits) issue(blockIdx.x + (long long)i * gridDim.x, i);
+    if (blockIdx.x + (long long)i * gridDim.x < nunits) issue(desc[i], i);
 
   float x[4][8];
   int it = 0;
@@ -411,7 +428,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   for (long long u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const int st = it % kQuantStages;
     if (!block_wait(b_base + 8 * st, (it / kQuantStages) & 1, ws.status)) { ok = false; break; }
-    const QUnit q = quant_unit(pb, ws, u);
+    const QUnit q = desc[st];
     const uint8_t *stage = sm_q + st * stage_bytes;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -421,9 +438,15 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
     }
-    __syncthreads();  // stage consumed: refill it with the unit after next
     const long long un = u + (long long)kQuantStages * gridDim.x;
-    if (un < nunits) issue(un, st);
+    if (threadIdx.x == 0 && un < nunits) desc[kQuantStages] = quant_unit(pb, ws, un);
+    __syncthreads();  // stage consumed; next descriptor visible
+    if (un < nunits) {
+      const QUnit qn = desc[kQuantStages];
+      issue(qn, st);
+      __syncthreads();  // every thread has its copy of qn before desc[st] changes
+      if (threadIdx.x == 0) desc[st] = qn;
+    }
 
     if (q.kind == 0) {
       // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
@@ -661,7 +684,9 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // quantize: persistent, 2 blocks per SM
-  const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 64 * 4;
+  // stages | output tile | 4 barriers | colsum[128] | chan[128] | scratch[72] | desc[stages + 1]
+  const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 72 * 4 +
+                        (kQuantStages + 1) * sizeof(QUnit);
   e = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
   if (e != cudaSuccess) return e;
   const int nKt = ws.Nkv_pad / kKVTile;
