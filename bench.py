@@ -327,7 +327,7 @@ def run_ours(args, w: Workload):
     peak8 = 2.0 * bf16_tflops  # 8-bit dense = 2 x bf16 dense (nominal 4.5 / 2.25 PFLOP/s)
     achieved = w.ops / (attn_ms * 1e-3) / 1e12
     value = replica_value(world, w.ops, step_ms)
-    kernels_per_step = 3 + (1 if w.smooth_q else 0)  # kv_stats, quantize, (delta_s), attention
+    kernels_per_step = 4 + (1 if w.smooth_q else 0)  # kv_stats, kv_finalize, quantize, (delta_s), attention
 
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,

@@ -10,16 +10,20 @@
 //   O += P8 v8                     fp32 accumulation, tensor cores (kind::f8f6f4)
 //   out = O * v_scale / l (+ mean_v), rounded to bf16 / fp16
 //
-// One CTA (192 threads) owns one query tile; two CTAs share an SM, so the
-// tensor core alternates between them while each runs its softmax.
+// One CTA (256 threads, two warpgroups) owns one query tile; two CTAs share
+// an SM, so the tensor core alternates between them while each runs its
+// softmax.  The helper warpgroup gives registers to the softmax warpgroup
+// (setmaxnreg).
 //   warp 0      TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ... into a
 //               3-stage shared-memory ring (order = MMA consumption order)
 //   warp 1      allocates 256 TMEM columns; lane 0 issues the MMAs:
 //               S_{j+1} = Q K_{j+1}^T as soon as softmax has read S_j, then
 //               O += P_j V_j once P_j is in shared memory
-//   warps 2-5   softmax: one query row per thread (TMEM lane), reads S with
+//   warps 2-3   idle
+//   warps 4-7   softmax: one query row per thread (TMEM lane), reads S with
 //               tcgen05.ld, writes P_j (swizzled, double-buffered) to shared
-//               memory, rescales its O row in TMEM when the max grows, and
+//               memory 32 keys at a time, rescales its O row in TMEM when the
+//               reference max moves (overlapped with the exponentials), and
 //               runs the epilogue
 // TMEM: S at columns [0,128), O at [128, 128 + D).
 // Causal tiles past the diagonal are skipped; keys >= Nkv and (causal)
@@ -28,6 +32,8 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+
+#include <cfloat>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -52,8 +58,15 @@ struct Cfg {
   static constexpr int kBarBytes = 256;
   static constexpr int kSmem = kOffBar + kBarBytes + 1024;   // +1024: base alignment slack
   static constexpr uint32_t kTmemCols = 256;
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 256;
 };
+
+// Register split of the attention CTA (256 threads launched at 128 registers
+// each): the helper warpgroup (TMA producer, MMA issuer, two idle warps)
+// gives registers back, the softmax warpgroup takes them.  56 * 128 + 200 *
+// 128 == 256 * 128, the block's whole allocation.
+constexpr uint32_t kLaunchRegs = 128, kHelperRegs = 56, kSoftmaxRegs = 200;
+static_assert(kHelperRegs * 128 + kSoftmaxRegs * 128 == kLaunchRegs * 256, "register split");
 
 // Barrier slots (8 bytes each) inside the barrier area.
 enum Bar {
@@ -73,37 +86,43 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int *st
   return __all_sync(0xffffffffu, ok);
 }
 
-// One query row's share of one KV tile (128 keys).  s[] holds the int32 S
-// row from TMEM; on return pk[] holds the 128 FP8 codes of P (key k in byte
-// k % 4 of pk[k / 4]) and lsum the sum of the unquantised probabilities.
-// m_used is the row's reference max (raised lazily, see kLazyLog2); alpha is
-// the factor O and l must be multiplied by (1 when m_used did not move).
-// Keys k >= lim are masked (only when kMasked).  Logits: x = S * c_half
-// (+ dsk with smoothed Q); the exponent t = x - (m_used - log2(224)) is one
-// fused fp32 op per key, as in the oracle.
+// One query row's share of one KV tile (128 keys), in two parts around the
+// lazy reference-max update.
+//
+// tile_max: s[] holds the int32 S row from TMEM and is biased in place to the
+// fp32 bit patterns of 1.5 * 2^23 + S (exact for |S| < 2^22, same order as
+// S); with smoothed Q it then holds the logits x = S * c_half + dsk.  Keys
+// k >= lim (only when kMasked) are set to -inf.  Returns the tile max of the
+// logits over the valid keys [0, lim) (-inf if none).
 template <bool kMasked, bool kSmoothQ>
-__device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float c1,
-                                             const float *dsk_tile, int lim, float &m_used,
-                                             float &alpha, bool &rescale, float &lsum,
-                                             uint32_t (&pk)[32]) {
-  // s[] is converted in place: from here on it holds fp32 bit patterns,
-  // S as float (exact), or the logits x with smoothed Q.
+__device__ __forceinline__ float tile_max(uint32_t (&s)[128], float c0, float c1,
+                                          const float *dsk_tile, int lim) {
+  constexpr float kBias = 12582912.0f;
 #define X(k) __uint_as_float(s[k])
 #pragma unroll
-  for (int k = 0; k < 128; ++k) s[k] = __float_as_uint(s32_to_f32_exact(s[k]));
+  for (int k = 0; k < 128; ++k) s[k] += 0x4B400000u;
   if (kSmoothQ) {
+    const float2 nb = make_float2(-kBias, -kBias);
 #pragma unroll
     for (int k = 0; k < 128; k += 4) {
       const float4 d4 = __ldg(reinterpret_cast<const float4 *>(dsk_tile + k));
       const float c = k < 64 ? c0 : c1;
-      s[k] = __float_as_uint(__fmaf_rn(X(k), c, d4.x));
-      s[k + 1] = __float_as_uint(__fmaf_rn(X(k + 1), c, d4.y));
-      s[k + 2] = __float_as_uint(__fmaf_rn(X(k + 2), c, d4.z));
-      s[k + 3] = __float_as_uint(__fmaf_rn(X(k + 3), c, d4.w));
+      const float2 c2 = make_float2(c, c);
+      const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(X(k), X(k + 1)), nb), c2, make_float2(d4.x, d4.y));
+      const float2 x23 = __ffma2_rn(__fadd2_rn(make_float2(X(k + 2), X(k + 3)), nb), c2, make_float2(d4.z, d4.w));
+      s[k] = __float_as_uint(x01.x);
+      s[k + 1] = __float_as_uint(x01.y);
+      s[k + 2] = __float_as_uint(x23.x);
+      s[k + 3] = __float_as_uint(x23.y);
     }
   }
-  // ---- tile max over valid keys (per 64-key half before scaling); eight
-  // independent 3-input max chains keep the dependency depth at 8
+  // keys k >= lim become -inf in place: they drop out of the max here and
+  // give 2^-inf = 0 in tile_exp
+  if (kMasked) {
+#pragma unroll
+    for (int k = 0; k < 128; ++k) s[k] = k < lim ? s[k] : 0xFF800000u;
+  }
+  // eight independent 3-input max chains keep the dependency depth at 8
   float h[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) h[q] = -INFINITY;
@@ -112,71 +131,99 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&s)[128], float c0, float
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int k0 = k + 2 * q, k1 = k0 + 64;
-      if (kMasked) {
-        h[q] = fmax3(h[q], k0 < lim ? X(k0) : -INFINITY, k0 + 1 < lim ? X(k0 + 1) : -INFINITY);
-        h[q + 4] = fmax3(h[q + 4], k1 < lim ? X(k1) : -INFINITY, k1 + 1 < lim ? X(k1 + 1) : -INFINITY);
-      } else {
-        h[q] = fmax3(h[q], X(k0), X(k0 + 1));
-        h[q + 4] = fmax3(h[q + 4], X(k1), X(k1 + 1));
-      }
+      h[q] = fmax3(h[q], X(k0), X(k0 + 1));
+      h[q + 4] = fmax3(h[q + 4], X(k1), X(k1 + 1));
     }
   }
   const float h0 = fmaxf(h[0], h[1]), h1 = fmaxf(h[2], h[3]);
   const float h2 = fmaxf(h[4], h[5]), h3 = fmaxf(h[6], h[7]);
   const float lo = fmaxf(h0, h1), hi = fmaxf(h2, h3);
-  float m_tile;
-  if (kSmoothQ) {
-    m_tile = fmaxf(lo, hi);
-  } else {
-    // max_j fl(S_j * c) == fl(max_j S_j * c) since c >= 0
-    m_tile = fmaxf(lo == -INFINITY ? -INFINITY : __fmul_rn(lo, c0),
-                   hi == -INFINITY ? -INFINITY : __fmul_rn(hi, c1));
-  }
-  // ---- lazy reference max
-  alpha = 1.f;
-  rescale = false;
-  if (m_tile != -INFINITY && (m_used == -INFINITY || m_tile > __fadd_rn(m_used, kLazyLog2))) {
-    if (m_used != -INFINITY) {
-      alpha = ex2_approx(__fsub_rn(m_used, m_tile));
-      rescale = true;
-    } else {
-      alpha = 0.f;
-    }
-    m_used = m_tile;
-  }
-  const float nmb = m_used == -INFINITY ? 0.f : -__fsub_rn(m_used, kLog2P8Scale);
-  // ---- probabilities, their sum, FP8 codes
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  if (kSmoothQ) return fmaxf(lo, hi);
+  // max_j fl(S_j * c) == fl(max_j S_j * c) since c >= 0; the biased max
+  // minus the bias is max_j S_j exactly
+  return fmaxf(lo == -INFINITY ? -INFINITY : __fmul_rn(__fsub_rn(lo, kBias), c0),
+               hi == -INFINITY ? -INFINITY : __fmul_rn(__fsub_rn(hi, kBias), c1));
+#undef X
+}
+
+// tile_exp: probabilities 2^(x - m_used + log2 224) of the valid keys, their
+// sum (returned) and their FP8 codes, stored to this row of the swizzled P
+// buffer 32 keys at a time.  With `rescale` (warp-uniform) the O row is
+// multiplied by `alpha` (1 for rows whose reference max did not move) in
+// 32-column TMEM chunks, chunk c's load in flight behind the exponentials of
+// keys 32 (c + 1) .. 32 (c + 1) + 31.  Pairs of keys go through f32x2 ops; every lane of a packed
+// op rounds like its scalar counterpart.
+template <int D, bool kSmoothQ>
+__device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], float c0, float c1, float nmb,
+                                          uint8_t *prow_base, int row, bool rescale, float alpha,
+                                          uint32_t tO) {
+  constexpr float kBias = 12582912.0f;
+  constexpr int kChunks = D / 32;
+#define X(k) __uint_as_float(s[k])
+  uint32_t o[32];
+  float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
+  const float2 nmb2 = make_float2(nmb, nmb), nb2 = make_float2(-kBias, -kBias);
+  const float2 a2 = make_float2(alpha, alpha);
+  // A scale product of exactly 0 means an all-zero Q or K block, so S = 0
+  // there; the smallest normal float in its place leaves S * c = 0 and keeps
+  // masked keys at -inf * c = -inf instead of NaN.
+  const float c0e = c0 == 0.f ? FLT_MIN : c0, c1e = c1 == 0.f ? FLT_MIN : c1;
+  const float2 c02 = make_float2(c0e, c0e), c12 = make_float2(c1e, c1e);
 #pragma unroll
-  for (int k = 0; k < 128; k += 4) {
-    float t0, t1, t2, t3;
-    if (kSmoothQ) {
-      t0 = __fadd_rn(X(k), nmb);
-      t1 = __fadd_rn(X(k + 1), nmb);
-      t2 = __fadd_rn(X(k + 2), nmb);
-      t3 = __fadd_rn(X(k + 3), nmb);
-    } else {
-      const float c = k < 64 ? c0 : c1;
-      t0 = __fmaf_rn(X(k), c, nmb);
-      t1 = __fmaf_rn(X(k + 1), c, nmb);
-      t2 = __fmaf_rn(X(k + 2), c, nmb);
-      t3 = __fmaf_rn(X(k + 3), c, nmb);
+  for (int sec = 0; sec < 4; ++sec) {
+    // O chunk sec - 1 is rescaled while the exponentials of keys 32 sec ..
+    // 32 sec + 31 are computed (register pressure peaks in section 0)
+    const int ch = sec - 1;
+    if (ch >= 0 && ch < kChunks && rescale) tmem_ld32_issue(tO + 32 * ch, o);
+    uint32_t pk[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int k = 32 * sec + 4 * q;
+      float2 t01, t23;
+      const float2 x01 = make_float2(X(k), X(k + 1)), x23 = make_float2(X(k + 2), X(k + 3));
+      if (kSmoothQ) {
+        t01 = __fadd2_rn(x01, nmb2);
+        t23 = __fadd2_rn(x23, nmb2);
+      } else {
+        const float2 c2 = k < 64 ? c02 : c12;
+        t01 = __ffma2_rn(__fadd2_rn(x01, nb2), c2, nmb2);
+        t23 = __ffma2_rn(__fadd2_rn(x23, nb2), c2, nmb2);
+      }
+      const float2 p01 = make_float2(ex2_approx(t01.x), ex2_approx(t01.y));
+      const float2 p23 = make_float2(ex2_approx(t23.x), ex2_approx(t23.y));
+      acc01 = __fadd2_rn(acc01, p01);
+      acc23 = __fadd2_rn(acc23, p23);
+      pk[q] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
     }
-    if (kMasked) {
-      t0 = k < lim ? t0 : -INFINITY;
-      t1 = k + 1 < lim ? t1 : -INFINITY;
-      t2 = k + 2 < lim ? t2 : -INFINITY;
-      t3 = k + 3 < lim ? t3 : -INFINITY;
+    // keys 32 sec .. 32 sec + 31 are the 16-byte units 2 sec and 2 sec + 1 of the row
+    *reinterpret_cast<uint4 *>(prow_base + swz_offset(row, 32 * sec, 128)) =
+        make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<uint4 *>(prow_base + swz_offset(row, 32 * sec + 16, 128)) =
+        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    if (ch >= 0 && ch < kChunks && rescale) {
+      tmem_ld32_wait(o);
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+        o[e] = __float_as_uint(o2.x);
+        o[e + 1] = __float_as_uint(o2.y);
+      }
+      tmem_st32_issue(tO + 32 * ch, o);
     }
-    const float p0 = ex2_approx(t0), p1 = ex2_approx(t1);
-    const float p2 = ex2_approx(t2), p3 = ex2_approx(t3);
-    a0 += p0;
-    a1 += p1;
-    a2 += p2;
-    a3 += p3;
-    pk[k / 4] = e4m3x4(p0, p1, p2, p3);
   }
-  lsum = (a0 + a1) + (a2 + a3);
+  if (kChunks == 4 && rescale) {
+    tmem_ld32_issue(tO + 96, o);
+    tmem_ld32_wait(o);
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const float2 o2 = __fmul2_rn(make_float2(__uint_as_float(o[e]), __uint_as_float(o[e + 1])), a2);
+      o[e] = __float_as_uint(o2.x);
+      o[e + 1] = __float_as_uint(o2.y);
+    }
+    tmem_st32_issue(tO + 96, o);
+  }
+  if (rescale) tmem_st_wait();
+  return (acc01.x + acc01.y) + (acc23.x + acc23.y);
 #undef X
 }
 
@@ -185,7 +232,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
 }
 
 template <int D, bool kSmoothQ>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __maxnreg__(128)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Problem pb, const Workspace ws) {
   using C = Cfg<D>;
@@ -234,6 +281,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *(volatile int *)status != 0;  // an earlier CTA already failed
 
+  if (warp < 4) {
+  reg_dealloc<kHelperRegs>();
   if (warp == 0) {
     // ================================================= TMA producer
     if (lane == 0 && !skip_all) {
@@ -322,7 +371,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mma_commit(bar(kBarFinal));
       mbar_wait(bar(kBarFinal), 0, status, false);
     }
+  }
   } else {
+    reg_alloc<kSoftmaxRegs>();
     // ================================================= softmax / correction / epilogue
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int row = 32 * wq + lane;          // row within the query tile
@@ -334,14 +385,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float *dsk = kSmoothQ ? ws.dsk + ((long long)bh * nq + qt) * ws.Nkv_pad : nullptr;
     float m_run = -INFINITY, l = 0.f;
     bool ok = !skip_all;
+    float ks0 = ksc[0], ks1 = ksc[1];   // K block scales of the tile, one tile ahead
     for (int j = 0; ok && j < T; ++j) {
       const int kb = j * kKVTile;
-      const float c0 = __fmul_rn(__fmul_rn(qs, ksc[2 * j]), pb.K2);
-      const float c1 = __fmul_rn(__fmul_rn(qs, ksc[2 * j + 1]), pb.K2);
+      const float c0 = __fmul_rn(__fmul_rn(qs, ks0), pb.K2);
+      const float c1 = __fmul_rn(__fmul_rn(qs, ks1), pb.K2);
+      if (j + 1 < T) {
+        ks0 = ksc[2 * j + 2];
+        ks1 = ksc[2 * j + 3];
+      }
       if (!warp_wait(bar(kBarSFull), j & 1, status)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[128];
-      tmem_ld128(tS, s);
+      tmem_ld64x2(tS, s);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(kBarSEmpty));
@@ -349,56 +405,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // valid keys of this tile for this row form the prefix [0, lim)
       int lim = min(kKVTile, pb.Nkv - kb);
       if (pb.is_causal) lim = min(lim, i - kb + 1);
+      const bool masked = lim < kKVTile;
       const float *dsk_tile = kSmoothQ ? dsk + kb : nullptr;
-      uint32_t pk[32];
-      float alpha, lsum;
-      bool need;
-      if (lim >= kKVTile)
-        softmax_tile<false, kSmoothQ>(s, c0, c1, dsk_tile, lim, m_run, alpha, need, lsum, pk);
-      else
-        softmax_tile<true, kSmoothQ>(s, c0, c1, dsk_tile, lim, m_run, alpha, need, lsum, pk);
-      l = __fmaf_rn(l, alpha, lsum);
-
-      // P_j -> shared buffer j & 1, once P V_{j-2} has finished reading it
-      if (j >= 2 && !warp_wait(bar(kBarPVDone + (j & 1)), ((j - 2) >> 1) & 1, status)) {
-        ok = false;
-        break;
+      const float m_tile = masked ? tile_max<true, kSmoothQ>(s, c0, c1, dsk_tile, lim)
+                                  : tile_max<false, kSmoothQ>(s, c0, c1, dsk_tile, lim);
+      // lazy reference max: raised (to the tile max) only when the tile max
+      // exceeds it by more than kLazyLog2
+      float alpha = 1.f;
+      bool need = false;
+      if (m_tile != -INFINITY && (m_run == -INFINITY || m_tile > __fadd_rn(m_run, kLazyLog2))) {
+        if (m_run != -INFINITY) {
+          alpha = ex2_approx(__fsub_rn(m_run, m_tile));
+          need = true;
+        } else {
+          alpha = 0.f;
+        }
+        m_run = m_tile;
       }
-      uint8_t *pbuf = smem + C::kOffP + (j & 1) * C::kPBytes;
-#pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4 *>(pbuf + swz_offset(row, 16 * cc, 128)) =
-            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-
-      // rescale this row of O when its reference max moved (after P V_{j-1} is done)
-      if (__any_sync(0xffffffffu, need)) {
+      const float nmb = m_run == -INFINITY ? 0.f : -__fsub_rn(m_run, kLog2P8Scale);
+      const bool rescale = __any_sync(0xffffffffu, need);
+      // P_j goes to shared buffer j & 1, free once P V_{j-2} is done; a
+      // rescale of O needs P V_{j-1} done, which implies P V_{j-2}
+      if (rescale) {
         if (!warp_wait(bar(kBarPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1, status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // the whole O row in one TMEM round trip
-        uint32_t r[D];
-        if constexpr (D == 128) {
-          tmem_ld128(tO, r);
-        } else if constexpr (D == 96) {
-          tmem_ld64(tO, r);
-          tmem_ld32(tO + 64, r + 64);
-        } else {
-          tmem_ld64(tO, r);
-        }
-        if (need)
-#pragma unroll
-          for (int e = 0; e < D; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-        if constexpr (D == 128) {
-          tmem_st128(tO, r);
-        } else if constexpr (D == 96) {
-          tmem_st64(tO, r);
-          tmem_st32(tO + 64, r + 64);
-        } else {
-          tmem_st64(tO, r);
-        }
+      } else if (j >= 2 && !warp_wait(bar(kBarPVDone + (j & 1)), ((j - 2) >> 1) & 1, status)) {
+        ok = false;
+        break;
       }
+      uint8_t *pbuf = smem + C::kOffP + (j & 1) * C::kPBytes;
+      const float a_row = need ? alpha : 1.f;
+      const float lsum = tile_exp<D, kSmoothQ>(s, c0, c1, nmb, pbuf, row, rescale, a_row, tO);
+      l = __fmaf_rn(l, alpha, lsum);
       // P stores visible to the tensor core (async proxy), TMEM writes ordered,
       // then P_j is handed to the MMA warp
       fence_proxy_async_smem();
@@ -636,6 +677,14 @@ template <int D, bool SQ>
 cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
                                 const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
   using C = Cfg<D>;
+  // The warpgroup register split adds up to exactly the launch allocation of
+  // kLaunchRegs per thread; with any other count the softmax warpgroup's
+  // setmaxnreg.inc could not be satisfied, so such a build is refused.
+  static const int launch_regs = [] {
+    cudaFuncAttributes fa{};
+    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, SQ>) == cudaSuccess ? fa.numRegs : -1;
+  }();
+  if (launch_regs != int(kLaunchRegs)) return cudaErrorInvalidKernelImage;
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
