@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define SAGE_ABI_VERSION 1
+#define SAGE_ABI_VERSION 2
 
 /* A CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st *sage_stream_t;
@@ -81,6 +81,10 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
  * comes from sage_workspace_size() and it must be 256-byte aligned.
  * Precondition of the exact fixed-point means: |x| * N < 2^39 for every
  * smoothed input x (e.g. |x| < 2^24 at N = 32768).  Inputs must be finite.
+ * fuse_q = 1 asks the whole pass (sage_attn_fwd and its two halves) to
+ * quantise Q inside the attention kernel instead of in the pre-pass; it
+ * applies without smooth_q and when the driver accepts a tensor map of q's
+ * strides, and gives the same q8, q_scale and output bit for bit.
  */
 typedef struct {
   const void *q, *k, *v;
@@ -90,6 +94,7 @@ typedef struct {
   int32_t layout;               /* sage_layout_t */
   int32_t dtype;                /* sage_dtype_t */
   int32_t is_causal, smooth_k, smooth_q, smooth_v;
+  int32_t fuse_q;               /* 0 or 1, see below */
   float sm_scale;
   void *workspace;
   size_t workspace_bytes;
@@ -130,8 +135,21 @@ sage_status_t sage_workspace_view(const sage_attn_params_t *p, sage_workspace_vi
 
 /* The whole pass: smoothing + quantisation pre-pass, then the attention
  * kernel, enqueued on `stream`.  Writes p->out.  Also resets the device
- * status word at its start. */
+ * status word at its start.  With fuse_q (see sage_attn_params_t) Q is
+ * quantised by the attention kernel (same codes and scale as the pre-pass
+ * would give; they are written to the workspace too). */
 sage_status_t sage_attn_fwd(const sage_attn_params_t *p, sage_stream_t stream);
+
+/* The two halves of sage_attn_fwd, exposed so that their device time can be
+ * measured apart; calling sage_attn_fwd_prepass and then
+ * sage_attn_fwd_attention with the same parameters and workspace is
+ * equivalent to sage_attn_fwd.  With fuse_q in effect the attention half
+ * quantises Q itself (from p->q, to the workspace's q8 / q_scale as well) and
+ * the pre-pass half quantises only K and V; otherwise the pre-pass half is
+ * sage_quantize and the attention half sage_attn_quantized.  The pre-pass
+ * half resets the device status word.  Errors as for sage_attn_fwd. */
+sage_status_t sage_attn_fwd_prepass(const sage_attn_params_t *p, sage_stream_t stream);
+sage_status_t sage_attn_fwd_attention(const sage_attn_params_t *p, sage_stream_t stream);
 
 /* Pre-pass only (steps 1-2): fills the workspace from q, k, v. */
 sage_status_t sage_quantize(const sage_attn_params_t *p, sage_stream_t stream);

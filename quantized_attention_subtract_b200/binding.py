@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
 EXPORTED = ["sage_abi_version", "sage_status_string", "sage_workspace_size", "sage_workspace_view",
             "sage_attn_fwd", "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
             "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop", "sage_debug_wait_timeout",
-            "sage_get_device_status", "sage_attn_fwd_noalloc"]
+            "sage_get_device_status", "sage_attn_fwd_noalloc", "sage_attn_fwd_prepass",
+            "sage_attn_fwd_attention"]
 
 
 class SageError(RuntimeError):
@@ -46,7 +47,7 @@ class Params(ctypes.Structure):
         ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("is_causal", ctypes.c_int32), ("smooth_k", ctypes.c_int32),
         ("smooth_q", ctypes.c_int32), ("smooth_v", ctypes.c_int32),
-        ("sm_scale", ctypes.c_float),
+        ("fuse_q", ctypes.c_int32), ("sm_scale", ctypes.c_float),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
     ]
 
@@ -80,7 +81,7 @@ def lib():
             L.sage_workspace_size.argtypes = [P, ctypes.POINTER(ctypes.c_size_t)]
             L.sage_workspace_view.argtypes = [P, ctypes.POINTER(WorkspaceView)]
             for f in (L.sage_attn_fwd, L.sage_quantize, L.sage_attn_quantized,
-                      L.sage_attn_fwd_noalloc):
+                      L.sage_attn_fwd_noalloc, L.sage_attn_fwd_prepass, L.sage_attn_fwd_attention):
                 f.argtypes = [P, vp]
             L.sage_debug_dump_s.argtypes = [P, i32, i32, i32, i32, vp, vp]
             L.sage_debug_pv.argtypes = [P, i32, i32, i32, vp, vp, vp]
@@ -120,7 +121,7 @@ def _dims(x: torch.Tensor, layout: str):
 
 
 def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scale=None,
-                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None) -> Params:
+                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None, fuse_q=False) -> Params:
     """Fill sage_attn_params_t from torch tensors (no copies, strides as given)."""
     B, Hq, Nq, D = _dims(q, tensor_layout)
     Bk, Hkv, Nkv, Dk = _dims(k, tensor_layout)
@@ -141,6 +142,7 @@ def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scal
     p.dtype = 0 if q.dtype == torch.float16 else 1
     p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
                                                        int(bool(smooth_q)), int(bool(smooth_v)))
+    p.fuse_q = int(bool(fuse_q))
     p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
     if workspace is not None:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
@@ -163,7 +165,7 @@ def alloc_workspace(p: Params, device) -> torch.Tensor:
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
              is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
              smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
-             workspace: torch.Tensor | None = None) -> torch.Tensor:
+             workspace: torch.Tensor | None = None, fuse_q: bool = False) -> torch.Tensor:
     """Quantized attention forward: INT8 Q K^T, FP8 P V, on the current CUDA stream.
 
     q: [B, Hq, Nq, D] ("HND") or [B, Nq, Hq, D] ("NHD"); k, v: same with Hkv, Nkv.
@@ -172,16 +174,17 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
     copy of one chunk, the kernels of the previous one and the device-to-host
     copy of the one before overlap; the returned host tensor is complete once
     the current stream has passed this call (pinned host tensors make the
-    copies asynchronous).
+    copies asynchronous).  fuse_q: quantise Q inside the attention kernel
+    instead of in the pre-pass (no effect with smooth_q; same results).
     """
     if not q.is_cuda:
         return _sageattn_host(q, k, v, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                              smooth_v, out)
+                              smooth_v, out, fuse_q)
     if not (k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be on the same device")
     dev_out = torch.empty_like(q) if out is None else out
     p = make_params(q, k, v, dev_out, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                    smooth_v)
+                    smooth_v, fuse_q=fuse_q)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     else:
@@ -209,7 +212,8 @@ def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int):
     return chunks
 
 
-def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out):
+def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out,
+                   fuse_q=False):
     dev = torch.device("cuda", torch.cuda.current_device())
     B, Hq, Nq, D = _dims(q, layout)
     _, Hkv, Nkv, _ = _dims(k, layout)
@@ -233,7 +237,7 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
     first = make_params(sl(qd, *chunks[0][:1], chunks[0][1] * group, chunks[0][2] * group),
                         sl(kd, *chunks[0]), sl(vd, *chunks[0]),
                         sl(od, chunks[0][0], chunks[0][1] * group, chunks[0][2] * group),
-                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, fuse_q=fuse_q)
     ws = alloc_workspace(first, dev)
     done_out = None
     for b, h0, h1 in chunks:
@@ -247,7 +251,8 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
             landed = torch.cuda.Event()
             landed.record(h2d)
         compute.wait_event(landed)
-        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v,
+                        fuse_q=fuse_q)
         need = workspace_bytes(p)
         if need > ws.numel():
             ws = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -287,6 +292,14 @@ def attn_quantized(p: Params, device) -> None:
 
 def attn_fwd(p: Params, device) -> None:
     _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(device)), "sage_attn_fwd")
+
+
+def attn_fwd_prepass(p: Params, device) -> None:
+    _check(lib().sage_attn_fwd_prepass(ctypes.byref(p), _stream(device)), "sage_attn_fwd_prepass")
+
+
+def attn_fwd_attention(p: Params, device) -> None:
+    _check(lib().sage_attn_fwd_attention(ctypes.byref(p), _stream(device)), "sage_attn_fwd_attention")
 
 
 def workspace_views(p: Params, workspace: torch.Tensor) -> dict:

@@ -227,11 +227,94 @@ __device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], float c0, fl
 #undef X
 }
 
+// Fused Q quantisation (no smoothing of Q), run by all 256 threads of the
+// CTA before the warp roles split: the CTA's 16-bit Q tile is in shared
+// memory at `qin` as D/32 boxes of [128 rows][32 channels] with the 64-byte
+// swizzle (rows past Nq are zero).  Thread (row, half) reads the half's
+// 16-channel units of its row, the eight warps agree on the block amax (one
+// CTA barrier), and every thread writes its units' INT8 codes into the
+// swizzled Q operand tile `sq` and into the workspace copy `q8_row` (half 1
+// also writes the zero padding units when D < Dp).  The same arithmetic as
+// the pre-pass: scale = amax / 127, code = rint(fl(x * (127 / amax))).
+// Returns the block scale.  With ok == false the tile is not read and the
+// codes are zero.
+template <int D>
+__device__ __forceinline__ float fused_quantize_q(const uint8_t *qin, uint8_t *sq, uint8_t *q8_row,
+                                                  float *xw, bool ok, bool bf16, int row, int half) {
+  constexpr int Dp = Cfg<D>::Dp, kMine = D / 32;  // 16-channel units per half row
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int u0 = half * kMine;
+  uint32_t w[8 * kMine];  // 16-bit channel pairs (channel 2i in the low half)
+#pragma unroll
+  for (int t = 0; t < kMine; ++t) {
+    const int u = u0 + t;  // unit u = chunks 2 (u % 2), +1 of box u / 2
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (ok) v = *reinterpret_cast<const uint4 *>(qin + 8192 * (u >> 1) + swz_offset(row, 32 * (u & 1) + 16 * c, 64));
+      w[8 * t + 4 * c] = v.x;
+      w[8 * t + 4 * c + 1] = v.y;
+      w[8 * t + 4 * c + 2] = v.z;
+      w[8 * t + 4 * c + 3] = v.w;
+    }
+  }
+  // |x| of a finite 16-bit float orders like its bit pattern with the sign
+  // cleared; four independent max chains
+  uint32_t m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8 * kMine; ++e) m4[e & 3] = __vmaxu2(m4[e & 3], w[e] & 0x7FFF7FFFu);
+  const uint32_t m2 = __vmaxu2(__vmaxu2(m4[0], m4[1]), __vmaxu2(m4[2], m4[3]));
+  const uint32_t mb = max(m2 & 0xFFFFu, m2 >> 16);
+  float amax = bf16 ? __uint_as_float(mb << 16) : __half2float(__ushort_as_half((unsigned short)mb));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if (lane == 0) xw[warp] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(fmaxf(xw[0], xw[1]), fmaxf(xw[2], xw[3])), fmaxf(fmaxf(xw[4], xw[5]), fmaxf(xw[6], xw[7])));
+  float scale = 0.f, inv = 0.f;
+  if (amax >= kTinyAmax) {
+    scale = __fdiv_rn(amax, 127.0f);
+    inv = __fdiv_rn(127.0f, amax);
+  }
+#pragma unroll
+  for (int t = 0; t < kMine; ++t) {
+    uint32_t cw[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t w0 = w[8 * t + 2 * q], w1 = w[8 * t + 2 * q + 1];
+      float2 x01, x23;
+      if (bf16) {
+        x01 = make_float2(__uint_as_float(w0 << 16), __uint_as_float(w0 & 0xFFFF0000u));
+        x23 = make_float2(__uint_as_float(w1 << 16), __uint_as_float(w1 & 0xFFFF0000u));
+      } else {
+        x01 = __half22float2(*reinterpret_cast<const __half2 *>(&w0));
+        x23 = __half22float2(*reinterpret_cast<const __half2 *>(&w1));
+      }
+      // scalar int8_bits: its separately rounded multiply and add must not be
+      // contracted into one fused multiply-add (packed f32x2 forms may be)
+      cw[q] = pack4_lo(int8_bits(x01.x, inv), int8_bits(x01.y, inv), int8_bits(x23.x, inv),
+                       int8_bits(x23.y, inv));
+    }
+    const int u = u0 + t;
+    const uint4 c4 = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    *reinterpret_cast<uint4 *>(sq + swz_offset(row, 16 * u, Dp)) = c4;
+    *reinterpret_cast<uint4 *>(q8_row + 16 * u) = c4;
+  }
+  if (half == 1) {
+#pragma unroll
+    for (int u = D / 16; u < Dp / 16; ++u) {
+      *reinterpret_cast<uint4 *>(sq + swz_offset(row, 16 * u, Dp)) = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4 *>(q8_row + 16 * u) = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+  return scale;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D, bool kSmoothQ>
+template <int D, bool kSmoothQ, bool kFuseQ>
 __global__ void __maxnreg__(128)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Problem pb, const Workspace ws) {
@@ -281,37 +364,91 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *(volatile int *)status != 0;  // an earlier CTA already failed
 
+  // ---- TMA issue state of the producer thread (thread 0).  Ring loads go in
+  // MMA consumption order K_0, K_1, V_0, K_2, V_1, ...; `n` counts the loads
+  // issued, `pos` the positions of that order already visited.
+  int n = 0, pos = 0, n_early = 0;
+  bool pok = true;
+  auto issue = [&](bool isK, int j) {
+    if (!pok) return;
+    const int st = n % C::kStages;
+    const uint32_t ph = (n / C::kStages) & 1;
+    if (!mbar_wait(bar(kBarEmpty + st), ph ^ 1, status)) { pok = false; return; }
+    const uint32_t dst = sRing + st * C::kStageBytes;
+    if (isK) {
+      mbar_arrive_expect_tx(bar(kBarFull + st), C::kKBytes);
+      tma_load_2d(dst, &tm_k, bar(kBarFull + st), 0, bhk * ws.Nkv_pad + j * kKVTile);
+    } else {
+      mbar_arrive_expect_tx(bar(kBarFull + st), C::kVBytes);
+      tma_load_2d(dst, &tm_v, bar(kBarFull + st), j * kKVTile, bhk * D);
+    }
+    ++n;
+  };
+  // visit the whole order; issue the positions in [n_early, limit)
+  auto issue_order = [&](int limit) {
+    pos = 0;
+    auto step = [&](bool isK, int j) {
+      if (pos >= n_early && pos < limit) issue(isK, j);
+      ++pos;
+    };
+    step(true, 0);
+    for (int j = 0; j < T && pos < limit; ++j) {
+      if (j + 1 < T) step(true, j + 1);
+      step(false, j);
+    }
+  };
+  if (threadIdx.x == 0 && !skip_all) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    if constexpr (kFuseQ) {
+      // the 16-bit Q tile into the P buffers (free until the first P_j):
+      // D/32 boxes of 32 channels x 128 rows, zero past Nq; then the first
+      // ring stages (fresh, no wait), all landing while Q is quantised
+      mbar_arrive_expect_tx(bar(kBarQ), 128 * D * 2);
+#pragma unroll
+      for (int bx = 0; bx < D / 32; ++bx) {
+        if (pb.q_map_hn)
+          tma_load_4d(sP + 8192 * bx, &tm_q, bar(kBarQ), 32 * bx, h, q0, b);
+        else
+          tma_load_4d(sP + 8192 * bx, &tm_q, bar(kBarQ), 32 * bx, q0, h, b);
+      }
+      issue_order(C::kStages);
+      n_early = n;
+    } else {
+      mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
+      tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+    }
+  }
+  float qs_fused = 0.f;
+  if constexpr (kFuseQ) {
+    // ---- every thread: quantise the Q tile (thread = (row, half)); the
+    // generic writes of the INT8 tile are made visible to the tensor core's
+    // async proxy before the barrier that precedes the first MMA
+    const bool qok = !skip_all && mbar_wait(bar(kBarQ), 0, status);
+    const int qrow = threadIdx.x & 127, qhalf = threadIdx.x >> 7;
+    float *xw = reinterpret_cast<float *>(smem + C::kOffBar + 8 * kNumBars + 16);
+    uint8_t *q8_row = reinterpret_cast<uint8_t *>(ws.q8) + ((long long)bh * ws.Nq_pad + q0 + qrow) * C::Dp;
+    qs_fused = fused_quantize_q<D>(smem + C::kOffP, smem + C::kOffQ, q8_row, xw, qok, pb.bf16 != 0,
+                                   qrow, qhalf);
+    if (qok && threadIdx.x == 0) ws.q_scale[(long long)bh * nq + qt] = qs_fused;
+    fence_proxy_async_smem();
+    __syncthreads();
+  }
+
   if (warp < 4) {
   reg_dealloc<kHelperRegs>();
   if (warp == 0) {
     // ================================================= TMA producer
     if (lane == 0 && !skip_all) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
-      tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
-      int n = 0;
-      bool ok = true;
-      auto issue = [&](bool isK, int j) {
-        if (!ok) return;
-        const int st = n % C::kStages;
-        const uint32_t ph = (n / C::kStages) & 1;
-        if (!mbar_wait(bar(kBarEmpty + st), ph ^ 1, status)) { ok = false; return; }
-        const uint32_t dst = sRing + st * C::kStageBytes;
-        if (isK) {
-          mbar_arrive_expect_tx(bar(kBarFull + st), C::kKBytes);
-          tma_load_2d(dst, &tm_k, bar(kBarFull + st), 0, bhk * ws.Nkv_pad + j * kKVTile);
-        } else {
-          mbar_arrive_expect_tx(bar(kBarFull + st), C::kVBytes);
-          tma_load_2d(dst, &tm_v, bar(kBarFull + st), j * kKVTile, bhk * D);
+      if constexpr (kFuseQ) {
+        issue_order(1 << 30);
+      } else {
+        issue(true, 0);
+        for (int j = 0; j < T; ++j) {
+          if (j + 1 < T) issue(true, j + 1);
+          issue(false, j);
         }
-        ++n;
-      };
-      issue(true, 0);
-      for (int j = 0; j < T; ++j) {
-        if (j + 1 < T) issue(true, j + 1);
-        issue(false, j);
       }
       // Before leaving, make sure every copy issued has landed (bounded).
       mbar_wait(bar(kBarQ), 0, status, false);
@@ -326,7 +463,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint32_t id_o = idesc_e4m3_f32(128, D);
       const uint64_t dQ = smem_desc_kmajor(sQ, C::Dp);
       int n = 0;
-      bool ok = mbar_wait(bar(kBarQ), 0, status);
+      // with fused Q the INT8 tile was published by the barrier above
+      bool ok = kFuseQ ? true : mbar_wait(bar(kBarQ), 0, status);
       auto wait_stage = [&]() -> uint32_t {
         const int st = n % C::kStages;
         if (ok && !mbar_wait(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
@@ -380,7 +518,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int i = q0 + row;                  // query index
     const uint32_t lane_off = uint32_t(32 * wq) << 16;
     const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + 128;
-    const float qs = ws.q_scale[(long long)bh * nq + qt];
+    const float qs = kFuseQ ? qs_fused : ws.q_scale[(long long)bh * nq + qt];
     const float *ksc = ws.k_scale + (long long)bhk * (ws.Nkv_pad / kKBlk);
     const float *dsk = kSmoothQ ? ws.dsk + ((long long)bh * nq + qt) * ws.Nkv_pad : nullptr;
     float m_run = -INFINITY, l = 0.f;
@@ -673,7 +811,7 @@ __global__ void __launch_bounds__(128, 1) mma_loop_kernel(int iters, int32_t *si
   }
 }
 
-template <int D, bool SQ>
+template <int D, bool SQ, bool FQ>
 cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
                                 const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
   using C = Cfg<D>;
@@ -682,14 +820,14 @@ cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CU
   // setmaxnreg.inc could not be satisfied, so such a build is refused.
   static const int launch_regs = [] {
     cudaFuncAttributes fa{};
-    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, SQ>) == cudaSuccess ? fa.numRegs : -1;
+    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, SQ, FQ>) == cudaSuccess ? fa.numRegs : -1;
   }();
   if (launch_regs != int(kLaunchRegs)) return cudaErrorInvalidKernelImage;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ, FQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(pb.B) * unsigned(pb.Hq) * unsigned(ws.nqb);
-  attn_fwd_kernel<D, SQ><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
+  attn_fwd_kernel<D, SQ, FQ><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
   return cudaGetLastError();
 }
 
@@ -705,8 +843,11 @@ __global__ void wait_timeout_kernel(int *status) {
 template <int D>
 cudaError_t launch_attention_d(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
                                const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
-  return pb.smooth_q ? launch_attention_dq<D, true>(pb, ws, tq, tk, tv, stream)
-                     : launch_attention_dq<D, false>(pb, ws, tq, tk, tv, stream);
+  // Q is fused only without Q smoothing (the smoothed path needs the
+  // pre-pass's block means and its Delta S rows)
+  if (pb.smooth_q) return launch_attention_dq<D, true, false>(pb, ws, tq, tk, tv, stream);
+  return pb.q_fused ? launch_attention_dq<D, false, true>(pb, ws, tq, tk, tv, stream)
+                    : launch_attention_dq<D, false, false>(pb, ws, tq, tk, tv, stream);
 }
 
 template <int D>

@@ -55,9 +55,28 @@ struct Problem {
   int is_causal, smooth_k, smooth_q, smooth_v;
   float sm_scale;
   float K2;  // fp32(sm_scale * fp32(log2 e))
+  // Q quantised inside the attention kernel (from the 16-bit input, through a
+  // 4-D tensor map) instead of by the pre-pass; the pre-pass then skips Q.
+  int q_fused;
+  int q_map_hn;  // tensor-map dimension order (D, Hq, Nq, B) instead of (D, Nq, Hq, B)
 };
 
 // Host-side launchers (defined in prepass.cu / attn_fwd.cu).
+// ---- INT8 codes (pre-pass and the attention kernel's fused Q path)
+constexpr float kTinyAmax = 0x1p-64f;  // blocks below this quantise to zero
+
+// INT8 code of x with reciprocal scale inv: rint(fl(x * inv)), round half to
+// even.  Adding 1.5 * 2^23 in fp32 rounds to an integer exactly that way and
+// leaves it (two's complement) in the low mantissa bits; |fl(x * inv)| is at
+// most 127 * (1 + 2^-24), so the code is always in [-127, 127].
+__device__ __forceinline__ uint32_t int8_bits(float x, float inv) {
+  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
+}
+// Pack the low bytes of four such words (first in bits [0, 8)).
+__device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t stream);
 cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
                              const CUtensorMap &tm_k, const CUtensorMap &tm_v, cudaStream_t stream);

@@ -34,7 +34,6 @@
 namespace sage {
 namespace {
 
-constexpr float kTinyAmax = 0x1p-64f;  // blocks below this quantise to zero
 
 __device__ __forceinline__ void load8(const uint16_t *p, int bf16, float (&x)[8]) {
   const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
@@ -319,17 +318,6 @@ __device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
   b = scratch[65];
 }
 
-// INT8 code of x with reciprocal scale inv: rint(fl(x * inv)), round half to
-// even.  Adding 1.5 * 2^23 in fp32 rounds to an integer exactly that way and
-// leaves it (two's complement) in the low mantissa bits; |fl(x * inv)| is at
-// most 127 * (1 + 2^-24), so the code is always in [-127, 127].
-__device__ __forceinline__ uint32_t int8_bits(float x, float inv) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
-}
-// Pack the low bytes of four such words (first in bits [0, 8)).
-__device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
 
 // Copy a finished [rows][row_bytes] tile from shared memory to a contiguous
 // global destination with 16-byte stores.
@@ -401,7 +389,8 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   QUnit *desc = reinterpret_cast<QUnit *>(scratch + 72);    // [stages + 1]
   const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
   const int nKt = ws.Nkv_pad / kKVTile;
-  const long long nunits = 2LL * pb.B * pb.Hkv * nKt + (long long)pb.B * pb.Hq * ws.nqb;
+  // Q blocks come last; they are skipped when the attention kernel quantises Q
+  const long long nunits = 2LL * pb.B * pb.Hkv * nKt + (pb.q_fused ? 0LL : (long long)pb.B * pb.Hq * ws.nqb);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQuantStages; ++i) mbar_init(b_base + 8 * i, 1);
     fence_mbar_init();
@@ -690,7 +679,7 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   e = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
   if (e != cudaSuccess) return e;
   const int nKt = ws.Nkv_pad / kKVTile;
-  const long long nblk = (long long)pb.B * pb.Hq * ws.nqb + 2LL * pb.B * pb.Hkv * nKt;
+  const long long nblk = (pb.q_fused ? 0LL : (long long)pb.B * pb.Hq * ws.nqb) + 2LL * pb.B * pb.Hkv * nKt;
   const unsigned g2 = (unsigned)std::min<long long>(nblk, 2LL * sms);
   quantize_kernel<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws);
   e = cudaGetLastError();

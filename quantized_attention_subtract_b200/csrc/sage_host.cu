@@ -43,7 +43,7 @@ sage_status_t check_shape(const sage_attn_params_t *p) {
   if (p->Hq % p->Hkv != 0) return SAGE_ERR_INVALID_ARG;
   if (p->Nq > 0 && p->Nkv < 1) return SAGE_ERR_INVALID_ARG;
   if (!is_flag(p->is_causal) || !is_flag(p->smooth_k) || !is_flag(p->smooth_q) ||
-      !is_flag(p->smooth_v))
+      !is_flag(p->smooth_v) || !is_flag(p->fuse_q))
     return SAGE_ERR_INVALID_ARG;
   if (!(p->sm_scale == p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
   // TMA row coordinates and kernel indices are 32-bit
@@ -236,6 +236,29 @@ struct Maps {
   CUtensorMap q, k, v;
 };
 
+// Tensor map of the caller's 16-bit Q for the attention kernel's fused
+// quantisation: dimensions (D, Nq, Hq, B), or (D, Hq, Nq, B) when the head
+// stride is the smaller one, so the strides increase; box 32 channels x 128
+// tokens (x 1 x 1), 64-byte swizzle, zero fill past Nq.  Returns false when
+// the driver rejects the strides (the caller then quantises Q in the
+// pre-pass instead).
+bool make_q_input_map(const Problem &pb, CUtensorMap *m, int *hn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const bool head_inner = pb.qs_h < pb.qs_n;
+  *hn = head_inner ? 1 : 0;
+  const cuuint64_t dims[4] = {cuuint64_t(pb.D), cuuint64_t(head_inner ? pb.Hq : pb.Nq),
+                              cuuint64_t(head_inner ? pb.Nq : pb.Hq), cuuint64_t(pb.B)};
+  const cuuint64_t strides[3] = {cuuint64_t(2 * (head_inner ? pb.qs_h : pb.qs_n)),
+                                 cuuint64_t(2 * (head_inner ? pb.qs_n : pb.qs_h)), cuuint64_t(2 * pb.qs_b)};
+  const cuuint32_t box[4] = {32, head_inner ? 1u : 128u, head_inner ? 128u : 1u, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, pb.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+            const_cast<uint16_t *>(pb.q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_maps(const sage_attn_params_t *p, const Workspace &ws, Maps &m) {
   const uint64_t BHq = uint64_t(p->B) * p->Hq, BHk = uint64_t(p->B) * p->Hkv;
   return make_map(&m.q, ws.q8, ws.Dp, BHq * ws.Nq_pad, ws.Dp, 128) &&
@@ -258,7 +281,13 @@ sage_status_t validate(const sage_attn_params_t *p, bool need_inputs, bool need_
   return check_device();
 }
 
-sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, bool attn) {
+// pre / attn: which half of the pass to enqueue.  whole_pass: the halves of
+// sage_attn_fwd, where Q is quantised inside the attention kernel when the
+// caller asks for it (fuse_q), Q is not smoothed and the driver accepts a
+// tensor map of the caller's Q; the separate pre-pass and attention calls
+// always go through the workspace.
+sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, bool attn,
+                  bool whole_pass) {
   // No queries: nothing to compute and no pointer is read (empty tensors
   // may have null data pointers).
   sage_status_t s = check_shape(p);
@@ -268,13 +297,25 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   s = validate(p, pre, attn, L);
   if (s != SAGE_OK) return s;
   const Workspace ws = make_workspace(p, L);
-  const Problem pb = make_problem(p);
+  Problem pb = make_problem(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // With fuse_q the whole pass quantises Q inside the attention kernel (it
+  // still writes q8 and q_scale to the workspace) and the pre-pass skips Q.
+  // The decision depends only on p, so both halves agree.
+  Maps m;
+  if (whole_pass && p->fuse_q && !p->smooth_q) {
+    int hn = 0;
+    if (make_q_input_map(pb, &m.q, &hn)) {
+      pb.q_fused = 1;
+      pb.q_map_hn = hn;
+    }
+  }
   if (pre && cudaMemsetAsync(ws.status, 0, sizeof(int), st) != cudaSuccess) return SAGE_ERR_CUDA;
   if (pre && launch_prepass(pb, ws, st) != cudaSuccess) return SAGE_ERR_CUDA;
   if (attn) {
-    Maps m;
+    CUtensorMap q_input = m.q;
     if (!make_maps(p, ws, m)) return SAGE_ERR_CUDA;
+    if (pb.q_fused) m.q = q_input;
     if (launch_attention(pb, ws, m.q, m.k, m.v, st) != cudaSuccess) return SAGE_ERR_CUDA;
   }
   return SAGE_OK;
@@ -357,7 +398,15 @@ sage_status_t sage_workspace_view(const sage_attn_params_t *p, sage_workspace_vi
 }
 
 sage_status_t sage_attn_fwd(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, true, true);
+  return run(p, stream, true, true, true);
+}
+
+sage_status_t sage_attn_fwd_prepass(const sage_attn_params_t *p, sage_stream_t stream) {
+  return run(p, stream, true, false, true);
+}
+
+sage_status_t sage_attn_fwd_attention(const sage_attn_params_t *p, sage_stream_t stream) {
+  return run(p, stream, false, true, true);
 }
 
 sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t stream) {
@@ -370,15 +419,15 @@ sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t s
   sage_attn_params_t q = *p;
   q.workspace = scratch;
   q.workspace_bytes = SAGE_NOALLOC_MAX_WORKSPACE_BYTES;
-  return run(&q, stream, true, true);
+  return run(&q, stream, true, true, true);
 }
 
 sage_status_t sage_quantize(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, true, false);
+  return run(p, stream, true, false, false);
 }
 
 sage_status_t sage_attn_quantized(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, false, true);
+  return run(p, stream, false, true, false);
 }
 
 sage_status_t sage_debug_dump_s(const sage_attn_params_t *p, int32_t b, int32_t h, int32_t qtile,

@@ -35,12 +35,12 @@ def to_device(bits: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
 class GpuRun:
     """Inputs on the device, the output, the workspace and its views."""
 
-    def __init__(self, w: Workload, q, k, v, run_attention: bool = True):
+    def __init__(self, w: Workload, q, k, v, run_attention: bool = True, fuse_q: bool = False):
         self.w = w
         self.q, self.k, self.v = (to_device(x, w.dtype) for x in (q, k, v))
         self.out = torch.empty_like(self.q)
         self.p = binding.make_params(self.q, self.k, self.v, self.out, w.layout, w.is_causal, None,
-                                     w.smooth_k, w.smooth_q, w.smooth_v)
+                                     w.smooth_k, w.smooth_q, w.smooth_v, fuse_q=fuse_q)
         self.ws = binding.alloc_workspace(self.p, self.q.device)
         if run_attention:
             binding.attn_fwd(self.p, self.q.device)
@@ -54,11 +54,11 @@ class GpuRun:
         return self.out.double().cpu().numpy()
 
 
-def run_both(w: Workload, seed=None):
+def run_both(w: Workload, seed=None, fuse_q: bool = False):
     q, k, v = generate(w, seed)
     pr = oracle_problem(w)
     pre = oracle.prepass(pr, q, k, v)
-    g = GpuRun(w, q, k, v)
+    g = GpuRun(w, q, k, v, fuse_q=fuse_q)
     return q, k, v, pr, pre, g
 
 

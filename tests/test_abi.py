@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert sorted(binding.EXPORTED) == names
-    assert L.sage_abi_version() == 1
+    assert L.sage_abi_version() == 2
 
 
 def test_status_strings():
@@ -118,3 +118,30 @@ def test_binding_raises_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(binding, "_lib", None)
     with pytest.raises(RuntimeError, match="CUDA library missing"):
         binding.lib()
+
+
+def test_python_mirrors_match_the_c_structs(tmp_path):
+    """binding.Params / WorkspaceView have the size and field offsets that a C
+    compiler gives sage_attn_params_t / sage_workspace_view_t from the header."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    hdr = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    mirrors = (("sage_attn_params_t", binding.Params), ("sage_workspace_view_t", binding.WorkspaceView))
+    lines = ['#include <stdio.h>', '#include "sage_b200.h"', "int main(void) {"]
+    for cname, py in mirrors:
+        lines.append(f'  printf("{cname} size %zu\\n", sizeof({cname}));')
+        for field, _ in py._fields_:
+            lines.append(f'  printf("{cname} {field} %zu\\n", offsetof({cname}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", hdr, str(src), "-o", str(exe)], check=True)
+    got = dict(l.rsplit(" ", 1) for l in subprocess.run([str(exe)], check=True, capture_output=True,
+                                                          text=True).stdout.splitlines())
+    for cname, py in mirrors:
+        assert int(got[f"{cname} size"]) == ctypes.sizeof(py), cname
+        for field, _ in py._fields_:
+            assert int(got[f"{cname} {field}"]) == getattr(py, field).offset, (cname, field)

@@ -12,8 +12,8 @@ import oracle
 from quantized_attention_subtract_b200 import binding, sageattn
 from quantized_attention_subtract_b200.workloads import generate, random_problem
 
-from _common import (EXACT_COS, EXACT_REL_L1, MIRROR_COS, MIRROR_MAX_ABS, GpuRun, compare_output,
-                     oracle_problem, run_both, to_device)
+from _common import (EXACT_COS, EXACT_REL_L1, MIRROR_COS, MIRROR_MAX_ABS, GpuRun,
+                     assert_prepass_bit_exact, compare_output, oracle_problem, run_both, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,15 +31,44 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("fuse_q", [False, True], ids=["prepass_q", "fused_q"])
 @pytest.mark.parametrize("case", CASES, ids=[str(i) for i in range(len(CASES))])
-def test_attention_matches_oracle(case):
+def test_attention_matches_oracle(case, fuse_q):
     flags = {k: v for k, v in case.items() if k in ("smooth_k", "smooth_q", "smooth_v", "is_causal")}
     w = random_problem(*case["args"], layout=case.get("layout", "HND"), dtype=case["dtype"],
                        seed=11, k_offset_sigma=5.0, **flags)
-    q, k, v, pr, pre, g = run_both(w)
+    q, k, v, pr, pre, g = run_both(w, fuse_q=fuse_q)
+    # every workspace output of the whole pass, including q8 / q_scale, which
+    # the attention kernel itself writes when it quantises Q (fuse_q)
+    assert_prepass_bit_exact(w, pre, g)
     r = compare_output(pr, pre, q, k, v, g, oracle.all_tiles(pr))
     assert r["max_abs_excess"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
     assert r["rel_l1_exact"] <= EXACT_REL_L1 and r["cos_exact"] >= EXACT_COS, r
+
+
+FUSED = [
+    dict(args=(2, 4, 2, 300, 520, 128), dtype="bf16", layout="HND"),
+    dict(args=(1, 4, 4, 200, 520, 96), dtype="fp16", layout="NHD", is_causal=True),
+    dict(args=(1, 2, 2, 129, 300, 64), dtype="bf16", layout="NHD"),
+]
+
+
+@pytest.mark.parametrize("case", FUSED, ids=[str(i) for i in range(len(FUSED))])
+def test_fused_q_matches_separate_prepass(case):
+    """The whole pass (Q quantised inside the attention kernel) and the pre-pass
+    followed by attention on the workspace give bit-identical outputs and the
+    same q8 / q_scale."""
+    flags = {k: v for k, v in case.items() if k == "is_causal"}
+    w = random_problem(*case["args"], layout=case["layout"], dtype=case["dtype"], seed=21, **flags)
+    q, k, v = generate(w)
+    fused = GpuRun(w, q, k, v, fuse_q=True)
+    sep = GpuRun(w, q, k, v, run_attention=False)
+    binding.attn_quantized(sep.p, sep.q.device)
+    torch.cuda.synchronize()
+    assert binding.device_status(sep.p) == 0
+    assert torch.equal(fused.out, sep.out)
+    for name in ("q8", "q_scale", "k8", "k_scale", "v8t", "v_scale"):
+        assert torch.equal(fused.views[name], sep.views[name]), name
 
 
 def test_public_api_matches_params_path_and_host_tensors():
