@@ -91,15 +91,22 @@ __device__ __forceinline__ void decode8(uint4 u, int bf16, float (&x)[8]) {
   }
 }
 
-// Issue the row copies of one unit: rows [0, nrows) of a tensor starting at
+// Issue the copies of one unit: rows [0, nrows) of a tensor starting at
 // `src` with element stride `stride` between rows go to `dst` (row pitch
-// `rowb` bytes).  Called by every thread; thread t copies row t.  Thread 0
-// arms the barrier with the unit's byte count.
+// `rowb` bytes).  Called by every thread.  Dense rows (stride == row length)
+// are one copy by thread 0; otherwise thread t copies row t (many small
+// copies are much slower than one large one).  Thread 0 arms the barrier
+// with the unit's byte count.
 __device__ __forceinline__ void issue_rows(uint32_t dst, const uint16_t *src, long long stride,
                                            int nrows, int rowb, uint32_t bar, bool arm,
                                            uint32_t total_bytes) {
   if (arm && threadIdx.x == 0) mbar_arrive_expect_tx(bar, total_bytes);
-  if (int(threadIdx.x) < nrows) bulk_load(dst + threadIdx.x * rowb, src + threadIdx.x * stride, rowb, bar);
+  if (stride * 2 == rowb) {
+    // rows back to back in memory (dense tokens): one copy of the whole run
+    if (threadIdx.x == 0 && nrows > 0) bulk_load(dst, src, uint32_t(nrows) * rowb, bar);
+  } else if (int(threadIdx.x) < nrows) {
+    bulk_load(dst + threadIdx.x * rowb, src + threadIdx.x * stride, rowb, bar);
+  }
 }
 
 // Block-wide bounded wait; every thread learns whether it succeeded.
@@ -146,13 +153,20 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
     const uint32_t dst = s_base + st * stage_bytes, bar = b_base + 8 * st;
     const uint32_t bytes = uint32_t(n) * rowb * (pb.smooth_k ? 2 : 1);
     if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, bytes);
-    if (pb.smooth_k && int(threadIdx.x) < n)
-      bulk_load(dst + threadIdx.x * rowb, pb.k + b * pb.ks_b + h * pb.ks_h + (j0 + threadIdx.x) * pb.ks_n,
-                rowb, bar);
-    if (int(threadIdx.x) >= 128 - n && threadIdx.x < 128) {
+    const uint16_t *ksrc = pb.k + b * pb.ks_b + h * pb.ks_h + j0 * pb.ks_n;
+    const uint16_t *vsrc = pb.v + b * pb.vs_b + h * pb.vs_h + j0 * pb.vs_n;
+    // dense tokens: one copy per tensor; otherwise one per row (K rows by
+    // threads 0.., V rows by threads ..127)
+    if (pb.ks_n == D) {
+      if (pb.smooth_k && threadIdx.x == 0) bulk_load(dst, ksrc, uint32_t(n) * rowb, bar);
+    } else if (pb.smooth_k && int(threadIdx.x) < n) {
+      bulk_load(dst + threadIdx.x * rowb, ksrc + threadIdx.x * pb.ks_n, rowb, bar);
+    }
+    if (pb.vs_n == D) {
+      if (threadIdx.x == 127) bulk_load(dst + kStatChunk * rowb, vsrc, uint32_t(n) * rowb, bar);
+    } else if (int(threadIdx.x) >= 128 - n && threadIdx.x < 128) {
       const int r = threadIdx.x - (128 - n);
-      bulk_load(dst + (kStatChunk + r) * rowb,
-                pb.v + b * pb.vs_b + h * pb.vs_h + (j0 + r) * pb.vs_n, rowb, bar);
+      bulk_load(dst + (kStatChunk + r) * rowb, vsrc + r * pb.vs_n, rowb, bar);
     }
   };
 
@@ -286,38 +300,42 @@ __global__ void kv_finalize_kernel(Problem pb, Workspace ws) {
   ws.v_inv[ci] = inv;
 }
 
-// Block-wide max of two values (one per K half, or the same value twice);
-// up to 32 warps.  Warp partials meet in shared memory, warp 0 reduces them
-// and broadcasts the result.
-__device__ __forceinline__ void block_max2(float &a, float &b, float *scratch) {
+// Block-wide max of two non-negative values with one barrier: warp maxima go
+// into slot[0..1] by integer atomicMax (non-negative floats order like their
+// bits).  The slots must hold 0 before the call and stay untouched until
+// every thread has read them.
+__device__ __forceinline__ void block_max2_atomic(float &a, float &b, unsigned *slot) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
     b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
   }
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32, nw = blockDim.x / 32;
-  if (lane == 0) {
-    scratch[warp] = a;
-    scratch[32 + warp] = b;
+  if ((threadIdx.x & 31) == 0) {
+    atomicMax(slot, __float_as_uint(a));
+    atomicMax(slot + 1, __float_as_uint(b));
   }
   __syncthreads();
-  if (warp == 0) {
-    float x = lane < nw ? scratch[lane] : 0.f, y = lane < nw ? scratch[32 + lane] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-      y = fmaxf(y, __shfl_xor_sync(0xffffffffu, y, o));
-    }
-    if (lane == 0) {
-      scratch[64] = x;
-      scratch[65] = y;
-    }
-  }
-  __syncthreads();
-  a = scratch[64];
-  b = scratch[65];
+  a = __uint_as_float(slot[0]);
+  b = __uint_as_float(slot[1]);
 }
 
+// INT8 codes of a thread's four rows (4 rg .. +3) x eight channels (8 c8 ..
+// +7) straight to a [128][Dp] tile in global memory; the 16 (D/8) threads of
+// a row write its D bytes contiguously, and threads c8 < (Dp - D) / 8 also
+// write the row's zero padding.
+__device__ __forceinline__ void store_codes(uint8_t *dst, int Dp, int D, int c8, int rg,
+                                            const float (&x)[4][8], float inv) {
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
+                                 int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
+    const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
+                                 int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
+    uint8_t *row = dst + (4 * rg + r) * Dp;
+    *reinterpret_cast<uint2 *>(row + 8 * c8) = make_uint2(w0, w1);
+    if (8 * c8 < Dp - D) *reinterpret_cast<uint2 *>(row + D + 8 * c8) = make_uint2(0u, 0u);
+  }
+}
 
 // Copy a finished [rows][row_bytes] tile from shared memory to a contiguous
 // global destination with 16-byte stores.
@@ -386,6 +404,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   unsigned long long *colsum = reinterpret_cast<unsigned long long *>(bars + 4);
   float *chan = reinterpret_cast<float *>(colsum + 128);
   float *scratch = chan + 128;                               // 66 floats
+  unsigned *mslot = reinterpret_cast<unsigned *>(scratch + 66);  // [2 parities][2]
   QUnit *desc = reinterpret_cast<QUnit *>(scratch + 72);    // [stages + 1]
   const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
   const int nKt = ws.Nkv_pad / kKVTile;
@@ -394,11 +413,15 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQuantStages; ++i) mbar_init(b_base + 8 * i, 1);
     fence_mbar_init();
+    for (int i = 0; i < 4; ++i) mslot[i] = 0u;
   }
   __syncthreads();
-  // Unit descriptors are decoded once, by thread 0, into shared memory:
-  // desc[st] describes the unit whose rows are in (or on their way into)
-  // stage st; desc[kQuantStages] is the next one to issue.
+  // Unit descriptors are decoded once, by thread 0, into a ring of
+  // kQuantStages + 1 shared slots: iteration it reads slot it % (S + 1) and
+  // thread 0 fills slot (it + S) % (S + 1) -- the slot of iteration it - 1,
+  // which every thread has finished reading by this iteration's first
+  // barrier.
+  constexpr int kSlots = kQuantStages + 1;
   auto issue = [&](const QUnit &q, int st) {
     issue_rows(s_base + st * stage_bytes, q.src, q.stride, q.nvalid, rowb, b_base + 8 * st, true,
                uint32_t(q.nvalid) * rowb);
@@ -407,6 +430,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
     for (int i = 0; i < kQuantStages; ++i)
       if (blockIdx.x + (long long)i * gridDim.x < nunits)
         desc[i] = quant_unit(pb, ws, blockIdx.x + (long long)i * gridDim.x);
+  static_assert(kQuantStages + 1 == kSlots, "descriptor ring");
   __syncthreads();
   for (int i = 0; i < kQuantStages; ++i)
     if (blockIdx.x + (long long)i * gridDim.x < nunits) issue(desc[i], i);
@@ -417,7 +441,14 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   for (long long u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
     const int st = it % kQuantStages;
     if (!block_wait(b_base + 8 * st, (it / kQuantStages) & 1, ws.status)) { ok = false; break; }
-    const QUnit q = desc[st];
+    const QUnit q = desc[it % kSlots];
+    // block-max slots: this unit uses parity it & 1; the other parity (last
+    // read in iteration it - 1) is cleared for the next unit
+    unsigned *mx = mslot + 2 * (it & 1);
+    if (threadIdx.x == 0) {
+      mslot[2 * ((it + 1) & 1)] = 0u;
+      mslot[2 * ((it + 1) & 1) + 1] = 0u;
+    }
     const uint8_t *stage = sm_q + st * stage_bytes;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -428,14 +459,10 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
         for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
     }
     const long long un = u + (long long)kQuantStages * gridDim.x;
-    if (threadIdx.x == 0 && un < nunits) desc[kQuantStages] = quant_unit(pb, ws, un);
+    QUnit *dn = desc + (it + kQuantStages) % kSlots;
+    if (threadIdx.x == 0 && un < nunits) *dn = quant_unit(pb, ws, un);
     __syncthreads();  // stage consumed; next descriptor visible
-    if (un < nunits) {
-      const QUnit qn = desc[kQuantStages];
-      issue(qn, st);
-      __syncthreads();  // every thread has its copy of qn before desc[st] changes
-      if (threadIdx.x == 0) desc[st] = qn;
-    }
+    if (un < nunits) issue(*dn, st);
 
     if (q.kind == 0) {
       // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
@@ -457,7 +484,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
           }
       // rows 0..63 belong to block 2 t, rows 64..127 to 2 t + 1
       float a0 = rg < 16 ? a : 0.f, a1 = rg < 16 ? 0.f : a;
-      block_max2(a0, a1, scratch);
+      block_max2_atomic(a0, a1, mx);
       float inv0 = 0.f, inv1 = 0.f, s0 = 0.f, s1 = 0.f;
       if (a0 >= kTinyAmax) {
         s0 = __fdiv_rn(a0, 127.0f);
@@ -472,21 +499,8 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
         ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 2 * q.t + 1] = s1;
       }
       const float inv = rg < 16 ? inv0 : inv1;
-      if (Dp != D)
-        for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
-          *reinterpret_cast<uint32_t *>(tile + o) = 0u;
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
-                                     int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
-        const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
-                                     int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
-        *reinterpret_cast<uint2 *>(tile + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
-      }
-      __syncthreads();
-      store_tile(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, tile,
-                 128 * Dp);
+      store_codes(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, Dp, D,
+                  c8, rg, x, inv);
     } else if (q.kind == 1) {
       // ---------------- V tile: V' = V - mean_v, FP8 per channel, transposed
       float mean[8], inv[8];
@@ -567,30 +581,18 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[r][e]));
-      block_max2(a, unused, scratch);
+      block_max2_atomic(a, unused, mx);
       float inv = 0.f, scale = 0.f;
       if (a >= kTinyAmax) {
         scale = __fdiv_rn(a, 127.0f);
         inv = __fdiv_rn(127.0f, a);
       }
       if (threadIdx.x == 0) ws.q_scale[(long long)q.bh * ws.nqb + q.t] = scale;
-      if (Dp != D)
-        for (int o = 4 * threadIdx.x; o < 128 * Dp; o += 4 * blockDim.x)
-          *reinterpret_cast<uint32_t *>(tile + o) = 0u;
-      __syncthreads();
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
-                                     int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
-        const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
-                                     int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
-        *reinterpret_cast<uint2 *>(tile + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
-      }
-      __syncthreads();
-      store_tile(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, tile,
-                 128 * Dp);
+      store_codes(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, Dp, D,
+                  c8, rg, x, inv);
     }
-    __syncthreads();  // output tile free for the next unit
+    // The V transpose tile is rewritten only after the next unit's first
+    // barrier, which every thread reaches after its reads of this one.
   }
   if (!ok) {
     // wait (bounded) for copies still in flight before leaving
