@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define SAGE_ABI_VERSION 2
+#define SAGE_ABI_VERSION 3
 
 /* A CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st *sage_stream_t;
@@ -98,6 +98,17 @@ typedef struct {
   float sm_scale;
   void *workspace;
   size_t workspace_bytes;
+  /* Variable-length batch (both null for the batched layout): host arrays of
+   * B + 1 non-decreasing token offsets starting at 0.  Sequence b owns
+   * tokens [cu_seqlens_q[b], cu_seqlens_q[b+1]) of q and out and tokens
+   * [cu_seqlens_kv[b], cu_seqlens_kv[b+1]) of k and v: the B sequences are
+   * packed along the token axis of one tensor per input, and the batch
+   * strides are ignored.  Nq and Nkv are then bounds on the sequence lengths
+   * (they size the workspace); a sequence with queries needs at least one
+   * key.  Each sequence is its own problem (its own smoothing means and V
+   * scales; causal masking top-left within it).  The arrays are copied
+   * during the call.  fuse_q has no effect here. */
+  const int32_t *cu_seqlens_q, *cu_seqlens_kv;
 } sage_attn_params_t;
 
 /* Where the quantised tensors live inside the workspace (tests, debugging).

@@ -253,3 +253,54 @@ def delta_s(pr: Problem, pre: dict, b: int, h: int, qt: int) -> np.ndarray:
     out = np.zeros(pr.Nkv, np.float64)
     lib.oracle_delta_s(ctypes.byref(pr._c()), _ptr(mq), _ptr(kp), _ptr(out))
     return out
+
+
+def varlen_attention(Hq: int, Hkv: int, D: int, cu_q, cu_kv, q: np.ndarray, k: np.ndarray,
+                     v: np.ndarray, dtype: str = "fp16", is_causal: bool = False,
+                     smooth_k: bool = True, smooth_q: bool = False, smooth_v: bool = False,
+                     sm_scale: float | None = None, with_uncertainty: bool = False,
+                     exact: bool = False) -> dict:
+    """A variable-length batch of packed sequences ("variable sequence lengths
+    per batch", sageattention package page): sequence b is rows
+    cu_q[b] .. cu_q[b+1] of q [total_q, Hq, D] attending to rows
+    cu_kv[b] .. cu_kv[b+1] of k, v [total_kv, Hkv, D], and nothing else.
+    The pages fix no more than that; the reading taken is that each sequence
+    is its own problem -- its own smoothing means, scales and causal mask --
+    so this is the single-problem oracle run once per sequence.
+
+    Returns {"out": fp64 [total_q, Hq, D] (the mirror), "pre": [per-sequence
+    pre-pass dicts], "problems": [per-sequence Problem]}, plus "unc" and
+    "exact" of the output's shape when asked."""
+    cu_q, cu_kv = np.asarray(cu_q, np.int64), np.asarray(cu_kv, np.int64)
+    total_q = int(cu_q[-1])
+    res = {"out": np.zeros((total_q, Hq, D)), "pre": [], "problems": []}
+    if with_uncertainty:
+        res["unc"] = np.zeros_like(res["out"])
+    if exact:
+        res["exact"] = np.zeros_like(res["out"])
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_kv[b]), int(cu_kv[b + 1])
+        pr = Problem(B=1, Hq=Hq, Hkv=Hkv, Nq=q1 - q0, Nkv=k1 - k0, D=D, layout="NHD", dtype=dtype,
+                     is_causal=is_causal, smooth_k=smooth_k, smooth_q=smooth_q, smooth_v=smooth_v,
+                     sm_scale=sm_scale)
+        res["problems"].append(pr)
+        if q1 == q0:
+            res["pre"].append(None)
+            continue
+        qs, ks, vs = (np.ascontiguousarray(x[None]) for x in (q[q0:q1], k[k0:k1], v[k0:k1]))
+        pre = prepass(pr, qs, ks, vs)
+        res["pre"].append(pre)
+        tiles = all_tiles(pr)
+        parts = {"out": None, "unc": None, "exact": None}
+        if with_uncertainty:
+            parts["out"], parts["unc"] = attention_tiles(pr, pre, tiles, with_uncertainty=True)
+        else:
+            parts["out"] = attention_tiles(pr, pre, tiles)
+        if exact:
+            parts["exact"] = exact_attention_tiles(pr, qs, ks, vs, tiles)
+        for n, (_, h, t) in enumerate(tiles):
+            i0, i1 = t * QBLK, min(t * QBLK + QBLK, pr.Nq)
+            for name, arr in parts.items():
+                if arr is not None:
+                    res[name][q0 + i0:q0 + i1, h] = arr[n, :i1 - i0]
+    return res

@@ -11,6 +11,7 @@ import ctypes
 import os
 import threading
 
+import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +50,7 @@ class Params(ctypes.Structure):
         ("smooth_q", ctypes.c_int32), ("smooth_v", ctypes.c_int32),
         ("fuse_q", ctypes.c_int32), ("sm_scale", ctypes.c_float),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_kv", ctypes.c_void_p),
     ]
 
 
@@ -147,6 +149,78 @@ def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scal
     if workspace is not None:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
     return p
+
+
+def _host_offsets(cu) -> np.ndarray:
+    """Sequence offsets as a contiguous host int32 array."""
+    if isinstance(cu, torch.Tensor):
+        cu = cu.detach().to("cpu").numpy()
+    a = np.ascontiguousarray(np.asarray(cu), dtype=np.int32)
+    if a.ndim != 1 or a.size < 2:
+        raise ValueError("cu_seqlens must be 1-D with at least two entries")
+    return a
+
+
+def make_varlen_params(q, k, v, out, cu_seqlens_q, cu_seqlens_kv, max_seqlen_q=None,
+                       max_seqlen_kv=None, is_causal=False, sm_scale=None, smooth_k=True,
+                       smooth_q=False, smooth_v=False, workspace=None) -> Params:
+    """sage_attn_params_t for a variable-length batch: q [total_q, Hq, D],
+    k, v [total_kv, Hkv, D] (packed sequences), out like q; cu_seqlens_* hold
+    B + 1 offsets (host or device integer tensors / arrays, copied to host
+    int32)."""
+    cq, ck = _host_offsets(cu_seqlens_q), _host_offsets(cu_seqlens_kv)
+    if cq.size != ck.size:
+        raise ValueError("cu_seqlens_q and cu_seqlens_kv must have the same length")
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape:
+        raise ValueError("packed q, k, v must be [total, heads, head_dim]")
+    if q.shape[2] != k.shape[2]:
+        raise ValueError("q and k disagree on head_dim")
+    if q.dtype not in (torch.float16, torch.bfloat16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share dtype float16 or bfloat16")
+    lq, lk = np.diff(cq), np.diff(ck)
+    p = Params()
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.out = out.data_ptr() if out is not None else None
+    p.B, p.Hq, p.Hkv, p.D = cq.size - 1, q.shape[1], k.shape[1], q.shape[2]
+    p.Nq = int(max_seqlen_q) if max_seqlen_q is not None else int(max(lq.max(), 0))
+    p.Nkv = int(max_seqlen_kv) if max_seqlen_kv is not None else int(max(lk.max(), 0))
+    # NHD order (batch, token, head, channel); the batch stride is unused
+    for name, t in (("q_strides", q), ("k_strides", k), ("v_strides", v), ("o_strides", out)):
+        st = t.stride() if t is not None else (0, 0, 1)
+        getattr(p, name)[:] = [0, st[0], st[1], st[2]]
+    p.layout = 1
+    p.dtype = 0 if q.dtype == torch.float16 else 1
+    p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
+                                                       int(bool(smooth_q)), int(bool(smooth_v)))
+    p.fuse_q = 0
+    p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
+    p.cu_seqlens_q, p.cu_seqlens_kv = cq.ctypes.data, ck.ctypes.data
+    p._offsets = (cq, ck)  # the arrays must outlive every call made with p
+    if workspace is not None:
+        p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
+    return p
+
+
+def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q, cu_seqlens_k,
+                    max_seqlen_q: int | None = None, max_seqlen_k: int | None = None,
+                    is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
+                    smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Quantized attention over a variable-length batch of packed sequences on
+    the current CUDA stream: q [total_q, Hq, D], k, v [total_kv, Hkv, D] on
+    the device; sequence b owns tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]
+    of q (cu_seqlens_k of k, v) and attends only within itself.  Returns out
+    shaped like q."""
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    dev_out = torch.empty_like(q) if out is None else out
+    p = make_varlen_params(q, k, v, dev_out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                           is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+    ws = workspace if workspace is not None else alloc_workspace(p, q.device)
+    if workspace is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    attn_fwd(p, q.device)
+    return dev_out
 
 
 def workspace_bytes(p: Params) -> int:

@@ -343,9 +343,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int b = bh / pb.Hq, h = bh % pb.Hq;
   const int hk = h / (pb.Hq / pb.Hkv), bhk = b * pb.Hkv + hk;
   const int q0 = qt * kQBlk;
-  const int nkt_all = ws.Nkv_pad / kKVTile;
+  // this entry's lengths (a sequence of a variable-length batch may be
+  // shorter than the padded maximum: its surplus query tiles do nothing)
+  const int Nq_b = nq_of(pb, b), Nkv_b = nkv_of(pb, b);
+  if (q0 >= Nq_b) return;
+  const int nkt_all = (Nkv_b + kKVTile - 1) / kKVTile;
   int T = nkt_all;
-  if (pb.is_causal) T = min(nkt_all, min(q0 + kQBlk - 1, pb.Nq - 1) / kKVTile + 1);
+  if (pb.is_causal) T = min(nkt_all, min(q0 + kQBlk - 1, Nq_b - 1) / kKVTile + 1);
 
   if (threadIdx.x == 0) {
     // the softmax warps (4) arrive on S-empty and P-full; TMA bytes or a
@@ -541,7 +545,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (lane == 0) mbar_arrive(bar(kBarSEmpty));
 
       // valid keys of this tile for this row form the prefix [0, lim)
-      int lim = min(kKVTile, pb.Nkv - kb);
+      int lim = min(kKVTile, Nkv_b - kb);
       if (pb.is_causal) lim = min(lim, i - kb + 1);
       const bool masked = lim < kKVTile;
       const float *dsk_tile = kSmoothQ ? dsk + kb : nullptr;
@@ -593,7 +597,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float *vs = ws.v_scale + (long long)bhk * D;
       const float *mv = ws.mean_v + (long long)bhk * D;
       uint8_t *orow = reinterpret_cast<uint8_t *>(pb.out) +
-                      2 * (b * pb.os_b + h * pb.os_h + (long long)i * pb.os_n);
+                      2 * (o_off(pb, b) + h * pb.os_h + (long long)i * pb.os_n);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -615,7 +619,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             packed[e / 2] = *reinterpret_cast<const uint32_t *>(&v2);
           }
         }
-        if (i < pb.Nq) {
+        if (i < Nq_b) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             *reinterpret_cast<uint4 *>(orow + 64 * c + 16 * v4) =

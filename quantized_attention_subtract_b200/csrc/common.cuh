@@ -59,7 +59,33 @@ struct Problem {
   // 4-D tensor map) instead of by the pre-pass; the pre-pass then skips Q.
   int q_fused;
   int q_map_hn;  // tensor-map dimension order (D, Hq, Nq, B) instead of (D, Nq, Hq, B)
+  // Variable-length batches: batch entry b is sequence b with tokens
+  // [cu_q[b], cu_q[b+1]) of the packed q (and cu_kv of k, v); Nq / Nkv are
+  // then the maximum lengths and the batch strides are unused.  Null for
+  // the batched layout.  Device copies in the workspace.
+  const int *cu_q, *cu_kv;
 };
+
+// Per batch entry: query / key counts, and the element offset of (token 0,
+// head 0) of q, k, v and out.
+__device__ __forceinline__ int nq_of(const Problem &pb, int b) {
+  return pb.cu_q ? pb.cu_q[b + 1] - pb.cu_q[b] : pb.Nq;
+}
+__device__ __forceinline__ int nkv_of(const Problem &pb, int b) {
+  return pb.cu_kv ? pb.cu_kv[b + 1] - pb.cu_kv[b] : pb.Nkv;
+}
+__device__ __forceinline__ long long q_off(const Problem &pb, int b) {
+  return pb.cu_q ? (long long)pb.cu_q[b] * pb.qs_n : (long long)b * pb.qs_b;
+}
+__device__ __forceinline__ long long o_off(const Problem &pb, int b) {
+  return pb.cu_q ? (long long)pb.cu_q[b] * pb.os_n : (long long)b * pb.os_b;
+}
+__device__ __forceinline__ long long k_off(const Problem &pb, int b) {
+  return pb.cu_kv ? (long long)pb.cu_kv[b] * pb.ks_n : (long long)b * pb.ks_b;
+}
+__device__ __forceinline__ long long v_off(const Problem &pb, int b) {
+  return pb.cu_kv ? (long long)pb.cu_kv[b] * pb.vs_n : (long long)b * pb.vs_b;
+}
 
 // Host-side launchers (defined in prepass.cu / attn_fwd.cu).
 // ---- INT8 codes (pre-pass and the attention kernel's fused Q path)

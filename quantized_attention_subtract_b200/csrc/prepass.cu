@@ -144,17 +144,22 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
   auto unit_src = [&](long long u, int &bh, int &j0, int &n) {
     bh = int(u / nchunk);
     j0 = int(u % nchunk) * kStatChunk;
-    n = min(kStatChunk, pb.Nkv - j0);
+    n = min(kStatChunk, nkv_of(pb, bh / pb.Hkv) - j0);  // <= 0: past this sequence's end
   };
   auto issue = [&](long long u, int st) {
     int bh, j0, n;
     unit_src(u, bh, j0, n);
     const int b = bh / pb.Hkv, h = bh % pb.Hkv;
     const uint32_t dst = s_base + st * stage_bytes, bar = b_base + 8 * st;
+    if (n <= 0) {
+      // nothing to copy (past the sequence's end): complete the phase
+      if (threadIdx.x == 0) mbar_arrive(bar);
+      return;
+    }
     const uint32_t bytes = uint32_t(n) * rowb * (pb.smooth_k ? 2 : 1);
     if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, bytes);
-    const uint16_t *ksrc = pb.k + b * pb.ks_b + h * pb.ks_h + j0 * pb.ks_n;
-    const uint16_t *vsrc = pb.v + b * pb.vs_b + h * pb.vs_h + j0 * pb.vs_n;
+    const uint16_t *ksrc = pb.k + k_off(pb, b) + h * pb.ks_h + j0 * pb.ks_n;
+    const uint16_t *vsrc = pb.v + v_off(pb, b) + h * pb.vs_h + j0 * pb.vs_n;
     // dense tokens: one copy per tensor; otherwise one per row (K rows by
     // threads 0.., V rows by threads ..127)
     if (pb.ks_n == D) {
@@ -285,8 +290,13 @@ __global__ void kv_finalize_kernel(Problem pb, Workspace ws) {
   const int c = threadIdx.x;
   const long long ci = (long long)blockIdx.x * pb.D + c;
   if (c >= pb.D) return;
-  ws.mean_k[ci] = pb.smooth_k ? fixed_mean(ws.k_sum[ci], pb.Nkv) : 0.f;
-  const float mv = pb.smooth_v ? fixed_mean(ws.v_sum[ci], pb.Nkv) : 0.f;
+  const int n = nkv_of(pb, int(blockIdx.x) / pb.Hkv);
+  if (n <= 0) {  // a sequence without keys: nothing reads these
+    ws.mean_k[ci] = ws.mean_v[ci] = ws.v_scale[ci] = ws.v_inv[ci] = 0.f;
+    return;
+  }
+  ws.mean_k[ci] = pb.smooth_k ? fixed_mean(ws.k_sum[ci], n) : 0.f;
+  const float mv = pb.smooth_v ? fixed_mean(ws.v_sum[ci], n) : 0.f;
   ws.mean_v[ci] = mv;
   const float hi = __fsub_rn(key_float(ws.v_max[ci]), mv);
   const float lo = __fsub_rn(key_float(ws.v_min[ci]), mv);
@@ -371,12 +381,12 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
     q.b = q.bh / pb.Hkv;
     q.h = q.bh % pb.Hkv;
     q.r0 = q.t * kKVTile;
-    q.nvalid = max(0, min(kKVTile, pb.Nkv - q.r0));
+    q.nvalid = max(0, min(kKVTile, nkv_of(pb, q.b) - q.r0));
     if (q.kind == 0) {
-      q.src = pb.k + q.b * pb.ks_b + q.h * pb.ks_h + q.r0 * pb.ks_n;
+      q.src = pb.k + k_off(pb, q.b) + q.h * pb.ks_h + q.r0 * pb.ks_n;
       q.stride = pb.ks_n;
     } else {
-      q.src = pb.v + q.b * pb.vs_b + q.h * pb.vs_h + q.r0 * pb.vs_n;
+      q.src = pb.v + v_off(pb, q.b) + q.h * pb.vs_h + q.r0 * pb.vs_n;
       q.stride = pb.vs_n;
     }
   } else {
@@ -387,8 +397,8 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
     q.b = q.bh / pb.Hq;
     q.h = q.bh % pb.Hq;
     q.r0 = q.t * kQBlk;
-    q.nvalid = min(kQBlk, pb.Nq - q.r0);
-    q.src = pb.q + q.b * pb.qs_b + q.h * pb.qs_h + q.r0 * pb.qs_n;
+    q.nvalid = max(0, min(kQBlk, nq_of(pb, q.b) - q.r0));
+    q.src = pb.q + q_off(pb, q.b) + q.h * pb.qs_h + q.r0 * pb.qs_n;
     q.stride = pb.qs_n;
   }
   return q;
@@ -565,7 +575,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
         }
         __syncthreads();
         if (int(threadIdx.x) < D) {
-          const float m = fixed_mean((long long)colsum[threadIdx.x], q.nvalid);
+          const float m = q.nvalid > 0 ? fixed_mean((long long)colsum[threadIdx.x], q.nvalid) : 0.f;
           chan[threadIdx.x] = m;
           ws.mq[((long long)q.bh * ws.nqb + q.t) * D + threadIdx.x] = m;
         }
@@ -619,8 +629,8 @@ __global__ void __launch_bounds__(128) delta_s_kernel(Problem pb, Workspace ws) 
   for (int o = t; o < 128 * (D / 8); o += 128) {
     const int r = o / (D / 8), c8 = o % (D / 8), j = kt * 128 + r;
     float xv[8];
-    if (j < pb.Nkv) {
-      load8(pb.k + b * pb.ks_b + hk * pb.ks_h + (long long)j * pb.ks_n + 8 * c8, pb.bf16, xv);
+    if (j < nkv_of(pb, b)) {
+      load8(pb.k + k_off(pb, b) + hk * pb.ks_h + (long long)j * pb.ks_n + 8 * c8, pb.bf16, xv);
 #pragma unroll
       for (int e = 0; e < 8; ++e)
         xv[e] = __fsub_rn(xv[e], ws.mean_k[(long long)bhk * D + 8 * c8 + e]);

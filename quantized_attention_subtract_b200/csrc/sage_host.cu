@@ -27,7 +27,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct Layout {
   size_t off_q8, off_k8, off_v8t, off_qs, off_ks, off_vs, off_mk, off_mv, off_mq, off_dsk;
-  size_t off_ksum, off_vsum, off_vmax, off_vmin, off_vinv, off_status, total;
+  size_t off_ksum, off_vsum, off_vmax, off_vmin, off_vinv, off_status, off_cu, total;
   int Dp, Nq_pad, Nkv_pad, nqb, nkb;
 };
 
@@ -51,6 +51,24 @@ sage_status_t check_shape(const sage_attn_params_t *p) {
   if ((long long)p->B * p->Hq * nq_pad >= (1LL << 31)) return SAGE_ERR_UNSUPPORTED;
   if ((long long)p->B * p->Hkv * nkv_pad >= (1LL << 31)) return SAGE_ERR_UNSUPPORTED;
   if ((long long)p->B * p->Hkv * p->D >= (1LL << 31)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+bool is_varlen(const sage_attn_params_t *p) { return p->cu_seqlens_q != nullptr; }
+
+// Offsets of a variable-length batch (host arrays, read here): both or
+// neither given; start at 0, non-decreasing, each length within its bound,
+// at least one key for a sequence with queries.
+sage_status_t check_varlen(const sage_attn_params_t *p) {
+  if ((p->cu_seqlens_q == nullptr) != (p->cu_seqlens_kv == nullptr)) return SAGE_ERR_INVALID_ARG;
+  if (!is_varlen(p)) return SAGE_OK;
+  const int32_t *cq = p->cu_seqlens_q, *ck = p->cu_seqlens_kv;
+  if (cq[0] != 0 || ck[0] != 0) return SAGE_ERR_INVALID_ARG;
+  for (int b = 0; b < p->B; ++b) {
+    const long long lq = (long long)cq[b + 1] - cq[b], lk = (long long)ck[b + 1] - ck[b];
+    if (lq < 0 || lq > p->Nq || lk < 0 || lk > p->Nkv) return SAGE_ERR_INVALID_ARG;
+    if (lq > 0 && lk < 1) return SAGE_ERR_INVALID_ARG;
+  }
   return SAGE_OK;
 }
 
@@ -86,6 +104,7 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.off_vmin = take(BHk * D * sizeof(unsigned));
   L.off_vinv = take(BHk * D * sizeof(float));
   L.off_status = take(16);
+  L.off_cu = is_varlen(p) ? take(2 * (size_t(p->B) + 1) * sizeof(int32_t)) : 0;
   if (p->smooth_q) {
     L.off_mq = take(BHq * L.nqb * D * sizeof(float));
     L.off_dsk = take(BHq * L.nqb * size_t(L.Nkv_pad) * sizeof(float));
@@ -270,6 +289,7 @@ bool make_maps(const sage_attn_params_t *p, const Workspace &ws, Maps &m) {
 sage_status_t validate(const sage_attn_params_t *p, bool need_inputs, bool need_out, Layout &L) {
   sage_status_t s = check_shape(p);
   if (s != SAGE_OK) return s;
+  if ((s = check_varlen(p)) != SAGE_OK) return s;
   if (need_inputs) {
     if ((s = check_tensor(p->q, p->q_strides)) != SAGE_OK) return s;
     if ((s = check_tensor(p->k, p->k_strides)) != SAGE_OK) return s;
@@ -299,11 +319,21 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   const Workspace ws = make_workspace(p, L);
   Problem pb = make_problem(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (is_varlen(p)) {
+    // the kernels read the (validated) sequence offsets from the workspace
+    int32_t *cu = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(p->workspace) + L.off_cu);
+    const size_t n = (size_t(p->B) + 1) * sizeof(int32_t);
+    if (cudaMemcpyAsync(cu, p->cu_seqlens_q, n, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(cu + p->B + 1, p->cu_seqlens_kv, n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+    pb.cu_q = cu;
+    pb.cu_kv = cu + p->B + 1;
+  }
   // With fuse_q the whole pass quantises Q inside the attention kernel (it
   // still writes q8 and q_scale to the workspace) and the pre-pass skips Q.
   // The decision depends only on p, so both halves agree.
   Maps m;
-  if (whole_pass && p->fuse_q && !p->smooth_q) {
+  if (whole_pass && p->fuse_q && !p->smooth_q && !is_varlen(p)) {
     int hn = 0;
     if (make_q_input_map(pb, &m.q, &hn)) {
       pb.q_fused = 1;

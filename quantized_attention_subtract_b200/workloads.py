@@ -123,3 +123,23 @@ def random_problem(B, Hq, Hkv, Nq, Nkv, D, layout="HND", dtype="fp16", seed=0,
     """A small ad-hoc workload (tests)."""
     return Workload(f"adhoc_{B}_{Hq}_{Hkv}_{Nq}_{Nkv}_{D}", B, Hq, Hkv, Nq, Nkv, D, layout, dtype,
                     k_offset_sigma=k_offset_sigma, seed=seed, **flags)
+
+
+def generate_varlen(Hq: int, Hkv: int, D: int, lens_q, lens_kv, dtype: str = "fp16", seed: int = 0,
+                    k_offset_sigma: float = 3.0):
+    """A packed variable-length batch: returns (cu_q, cu_kv, q, k, v) with
+    q [sum(lens_q), Hq, D] and k, v [sum(lens_kv), Hkv, D] as uint16 bit
+    patterns (N(0,1); each sequence's K gets its own per-(head, channel)
+    offset N(0, k_offset_sigma)), and the int32 offsets."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens_q, lens_kv = np.asarray(lens_q, np.int64), np.asarray(lens_kv, np.int64)
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_kv = np.concatenate([[0], np.cumsum(lens_kv)]).astype(np.int32)
+    q = rng.standard_normal((int(cu_q[-1]), Hq, D), dtype=np.float32)
+    k = rng.standard_normal((int(cu_kv[-1]), Hkv, D), dtype=np.float32)
+    v = rng.standard_normal((int(cu_kv[-1]), Hkv, D), dtype=np.float32)
+    if k_offset_sigma > 0:
+        for b in range(len(lens_kv)):
+            off = rng.standard_normal((1, Hkv, D), dtype=np.float32) * np.float32(k_offset_sigma)
+            k[cu_kv[b]:cu_kv[b + 1]] += off
+    return cu_q, cu_kv, _to_bits(q, dtype), _to_bits(k, dtype), _to_bits(v, dtype)

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert sorted(binding.EXPORTED) == names
-    assert L.sage_abi_version() == 2
+    assert L.sage_abi_version() == 3
 
 
 def test_status_strings():
@@ -145,3 +145,49 @@ def test_python_mirrors_match_the_c_structs(tmp_path):
         assert int(got[f"{cname} size"]) == ctypes.sizeof(py), cname
         for field, _ in py._fields_:
             assert int(got[f"{cname} {field}"]) == getattr(py, field).offset, (cname, field)
+
+
+def _varlen_params(cu_q, cu_kv, **kw):
+    """Batched-shape params turned into a variable-length batch with host
+    offset arrays (kept alive on the returned object)."""
+    import numpy as np
+    cq, ck = np.asarray(cu_q, np.int32), np.asarray(cu_kv, np.int32)
+    p = _params(B=len(cq) - 1, **kw)
+    p.cu_seqlens_q, p.cu_seqlens_kv = cq.ctypes.data, ck.ctypes.data
+    p._keep = (cq, ck)
+    fake = 1 << 40
+    p.q = p.k = p.v = p.out = fake
+    p.workspace = fake
+    return p
+
+
+@pytest.mark.parametrize("cu_q,cu_kv,ok", [
+    ([0, 100, 256], [0, 200, 256], True),
+    ([0, 0, 256], [0, 0, 256], True),         # a sequence without queries needs no keys
+    ([1, 100, 256], [0, 200, 256], False),    # must start at 0
+    ([0, 200, 100], [0, 100, 200], False),    # decreasing
+    ([0, 100, 400], [0, 100, 200], False),    # longer than Nq = 256
+    ([0, 100, 200], [0, 0, 200], False),      # queries without keys
+])
+def test_varlen_offsets_checked_before_any_device_work(cu_q, cu_kv, ok):
+    p = _varlen_params(cu_q, cu_kv)
+    code, n = _ws_size(p)
+    assert code == 0
+    # one byte short: valid offsets get as far as the workspace check (and no
+    # further, so nothing is launched on any machine); invalid ones stop first
+    p.workspace_bytes = n - 1
+    assert _fwd(p) == (6 if ok else 1)
+
+
+def test_varlen_needs_both_offset_arrays():
+    p = _varlen_params([0, 100, 256], [0, 200, 256])
+    p.cu_seqlens_kv = None
+    p.workspace_bytes = _ws_size(p)[1] - 1
+    assert _fwd(p) == 1
+
+
+def test_varlen_workspace_holds_the_offsets():
+    batched = _params(B=2)
+    _, n0 = _ws_size(batched)
+    _, n1 = _ws_size(_varlen_params([0, 100, 256], [0, 200, 256]))
+    assert n1 > n0
