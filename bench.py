@@ -364,6 +364,111 @@ def run_ours(args, w: Workload):
         print(json.dumps(line), flush=True)
 
 
+# A variable-length batch (packed sequences): 16 sequences of H32 D128 bf16
+# whose query and key lengths are drawn uniformly from [256, 4096] (seeded),
+# non-causal, smooth_k.  No single configuration of the pages is variable
+# length; this stands in for their "variable sequence lengths per batch".
+VARLEN = dict(name="varlen_16seq_256to4096_h32_d128_bf16", nseq=16, H=32, D=128, dtype="bf16",
+              lo=256, hi=4096, seed=4)
+
+
+def run_varlen(args):
+    """`--varlen`: the same JSON line for the variable-length batch above
+    (one process, one GPU)."""
+    import torch
+    from quantized_attention_subtract_b200 import binding
+    from quantized_attention_subtract_b200.workloads import generate_varlen
+    c = VARLEN
+    rng = np.random.default_rng(c["seed"])
+    lq = rng.integers(c["lo"], c["hi"] + 1, c["nseq"])
+    lk = rng.integers(c["lo"], c["hi"] + 1, c["nseq"])
+    cu_q, cu_kv, q, k, v = generate_varlen(c["H"], c["H"], c["D"], lq, lk, c["dtype"], seed=c["seed"])
+    ops = float(4.0 * c["H"] * c["D"] * np.sum(lq.astype(np.float64) * lk))
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    to_dev = lambda x: torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+    out = torch.empty_like(qd)
+    p = binding.make_varlen_params(qd, kd, vd, out, cu_q, cu_kv)
+    ws = binding.alloc_workspace(p, dev)
+    stream = torch.cuda.current_stream(dev)
+    clk = ClockSampler(0)
+    clk.start()
+    for _ in range(args.warmup):
+        binding.attn_fwd(p, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clk.mark_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        binding.attn_fwd(p, dev)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk.mark_end()
+    step_ms = e0.elapsed_time(e1) / args.steps
+    evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(args.steps)]
+    for a_, b_, c_ in evs:
+        a_.record(stream)
+        binding.attn_fwd_prepass(p, dev)
+        b_.record(stream)
+        binding.attn_fwd_attention(p, dev)
+        c_.record(stream)
+    torch.cuda.synchronize(dev)
+    pre_ms = float(np.mean([x.elapsed_time(y) for x, y, _ in evs]))
+    attn_ms = float(np.mean([y.elapsed_time(z) for _, y, z in evs]))
+    clk.stop()
+    assert binding.device_status(p) == 0, "device status nonzero"
+    # end to end: inputs from pinned host buffers and the output back, per step
+    qh, kh, vh = (x.cpu().pin_memory() for x in (qd, kd, vd))
+    oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        binding.attn_fwd(p, dev)
+        oh.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    bf16_tflops, _, peak_src = _peaks()
+    peak8 = 2.0 * bf16_tflops
+    achieved = ops / (attn_ms * 1e-3) / 1e12
+    in_bytes = 2 * (qd.numel() + kd.numel() + vd.numel())
+    line = {
+        "metric": METRIC, "value": ops / (step_ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)",
+        "data": "synthetic",
+        "config": {"workload": c["name"], "sequences": c["nseq"], "Hq": c["H"], "Hkv": c["H"],
+                   "D": c["D"], "total_q": int(cu_q[-1]), "total_kv": int(cu_kv[-1]),
+                   "max_q": int(lq.max()), "max_kv": int(lk.max()), "layout": "packed [total, H, D]",
+                   "input_dtype": c["dtype"], "causal": False, "smooth_k": True,
+                   "parallelism": "replicas x1",
+                   "l2": f"inputs {in_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)"},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved, "peak": peak8,
+                     "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 x 2 (burst)", "attn_ms": attn_ms,
+                     "prepass_ms": pre_ms},
+        "e2e": {"value": ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": out.numel() * 2},
+        "clocks": clk.summary(),
+        "gpu_launches": 4 * args.steps,
+    }
+    if not args.no_cpu_baseline:
+        # the oracle on a bounded sample of the first sequence (a batched
+        # problem of its shape, inputs drawn the same way)
+        w0 = Workload(c["name"] + "_seq0", 1, c["H"], c["H"], int(lq[0]), int(lk[0]), c["D"], "HND",
+                      c["dtype"], k_offset_sigma=3.0, seed=c["seed"])
+        heads, tiles = _sample_size(w0, 12.0)
+        tops, dt, desc, threads = oracle_sample(w0, heads, tiles)
+        line["cpu_baseline"] = {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                                "sample": desc + f" ({dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -372,10 +477,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--varlen", action="store_true",
+                    help="time the variable-length batch instead of --workload (one GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = WORKLOADS[args.workload]
+    if args.varlen and args.impl == "ours":
+        run_varlen(args)
+        return
     if args.impl == "reference":
         run_reference(args, w)
     else:

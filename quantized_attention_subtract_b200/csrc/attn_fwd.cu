@@ -310,11 +310,37 @@ __device__ __forceinline__ float fused_quantize_q(const uint8_t *qin, uint8_t *s
   return scale;
 }
 
+// One K or V tile load of the producer thread into ring stage n % kStages
+// (after the stage's previous contents were consumed; bounded wait), in the
+// MMA's consumption order; advances n.  ok turns false on a timeout.
+template <int D>
+__device__ __forceinline__ void issue_kv(bool isK, int j, int &n, bool &ok, uint32_t bars,
+                                         uint32_t sRing, const CUtensorMap *tm_k,
+                                         const CUtensorMap *tm_v, int krow0, int vrow0, int *status) {
+  using C = Cfg<D>;
+  if (!ok) return;
+  const int st = n % C::kStages;
+  const uint32_t ph = (n / C::kStages) & 1;
+  if (!mbar_wait(bars + 8u * uint32_t(kBarEmpty + st), ph ^ 1, status)) {
+    ok = false;
+    return;
+  }
+  const uint32_t dst = sRing + st * C::kStageBytes, full = bars + 8u * uint32_t(kBarFull + st);
+  if (isK) {
+    mbar_arrive_expect_tx(full, C::kKBytes);
+    tma_load_2d(dst, tm_k, full, 0, krow0 + j * kKVTile);
+  } else {
+    mbar_arrive_expect_tx(full, C::kVBytes);
+    tma_load_2d(dst, tm_v, full, j * kKVTile, vrow0);
+  }
+  ++n;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
-template <int D, bool kSmoothQ, bool kFuseQ>
+template <int D, bool kSmoothQ, bool kFuseQ, bool kVarlen>
 __global__ void __maxnreg__(128)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const Problem pb, const Workspace ws) {
@@ -345,8 +371,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int q0 = qt * kQBlk;
   // this entry's lengths (a sequence of a variable-length batch may be
   // shorter than the padded maximum: its surplus query tiles do nothing)
-  const int Nq_b = nq_of(pb, b), Nkv_b = nkv_of(pb, b);
-  if (q0 >= Nq_b) return;
+  const int Nq_b = kVarlen ? nq_of(pb, b) : pb.Nq, Nkv_b = kVarlen ? nkv_of(pb, b) : pb.Nkv;
+  if (kVarlen && q0 >= Nq_b) return;
   const int nkt_all = (Nkv_b + kKVTile - 1) / kKVTile;
   int T = nkt_all;
   if (pb.is_causal) T = min(nkt_all, min(q0 + kQBlk - 1, Nq_b - 1) / kKVTile + 1);
@@ -368,47 +394,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const uint32_t tmem = *tmem_slot;
   const bool skip_all = *(volatile int *)status != 0;  // an earlier CTA already failed
 
-  // ---- TMA issue state of the producer thread (thread 0).  Ring loads go in
-  // MMA consumption order K_0, K_1, V_0, K_2, V_1, ...; `n` counts the loads
-  // issued, `pos` the positions of that order already visited.
-  int n = 0, pos = 0, n_early = 0;
-  bool pok = true;
-  auto issue = [&](bool isK, int j) {
-    if (!pok) return;
-    const int st = n % C::kStages;
-    const uint32_t ph = (n / C::kStages) & 1;
-    if (!mbar_wait(bar(kBarEmpty + st), ph ^ 1, status)) { pok = false; return; }
-    const uint32_t dst = sRing + st * C::kStageBytes;
-    if (isK) {
-      mbar_arrive_expect_tx(bar(kBarFull + st), C::kKBytes);
-      tma_load_2d(dst, &tm_k, bar(kBarFull + st), 0, bhk * ws.Nkv_pad + j * kKVTile);
-    } else {
-      mbar_arrive_expect_tx(bar(kBarFull + st), C::kVBytes);
-      tma_load_2d(dst, &tm_v, bar(kBarFull + st), j * kKVTile, bhk * D);
-    }
-    ++n;
-  };
-  // visit the whole order; issue the positions in [n_early, limit)
-  auto issue_order = [&](int limit) {
-    pos = 0;
-    auto step = [&](bool isK, int j) {
-      if (pos >= n_early && pos < limit) issue(isK, j);
-      ++pos;
-    };
-    step(true, 0);
-    for (int j = 0; j < T && pos < limit; ++j) {
-      if (j + 1 < T) step(true, j + 1);
-      step(false, j);
-    }
-  };
-  if (threadIdx.x == 0 && !skip_all) {
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    if constexpr (kFuseQ) {
+  // ---- producer (thread 0) state: with fused Q the first ring loads are
+  // issued before the roles split, so that they land while Q is quantised;
+  // n_carry of them, which the producer loop then skips
+  int n_carry = 0;
+  if constexpr (kFuseQ) {
+    if (threadIdx.x == 0 && !skip_all) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
       // the 16-bit Q tile into the P buffers (free until the first P_j):
-      // D/32 boxes of 32 channels x 128 rows, zero past Nq; then the first
-      // ring stages (fresh, no wait), all landing while Q is quantised
+      // D/32 boxes of 32 channels x 128 rows, zero past Nq
       mbar_arrive_expect_tx(bar(kBarQ), 128 * D * 2);
 #pragma unroll
       for (int bx = 0; bx < D / 32; ++bx) {
@@ -417,11 +413,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         else
           tma_load_4d(sP + 8192 * bx, &tm_q, bar(kBarQ), 32 * bx, q0, h, b);
       }
-      issue_order(C::kStages);
-      n_early = n;
-    } else {
-      mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
-      tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+      // the first stages (fresh: no wait) in consumption order K_0, K_1, V_0
+      bool ok = true;
+      issue_kv<D>(true, 0, n_carry, ok, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D, status);
+      if (T > 1) issue_kv<D>(true, 1, n_carry, ok, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D, status);
+      issue_kv<D>(false, 0, n_carry, ok, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D, status);
     }
   }
   float qs_fused = 0.f;
@@ -445,14 +441,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == 0) {
     // ================================================= TMA producer
     if (lane == 0 && !skip_all) {
-      if constexpr (kFuseQ) {
-        issue_order(1 << 30);
-      } else {
-        issue(true, 0);
-        for (int j = 0; j < T; ++j) {
-          if (j + 1 < T) issue(true, j + 1);
-          issue(false, j);
+      if constexpr (!kFuseQ) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
+        tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+      }
+      int n = n_carry;
+      bool ok = true;
+      // K_0, K_1, V_0, K_2, V_1, ... skipping the n_carry loads issued early
+      int pos = 0;
+      auto issue = [&](bool isK, int j) {
+        if constexpr (kFuseQ) {
+          if (pos++ < n_carry) return;
         }
+        issue_kv<D>(isK, j, n, ok, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D, status);
+      };
+      issue(true, 0);
+      for (int j = 0; j < T; ++j) {
+        if (j + 1 < T) issue(true, j + 1);
+        issue(false, j);
       }
       // Before leaving, make sure every copy issued has landed (bounded).
       mbar_wait(bar(kBarQ), 0, status, false);
@@ -597,7 +606,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const float *vs = ws.v_scale + (long long)bhk * D;
       const float *mv = ws.mean_v + (long long)bhk * D;
       uint8_t *orow = reinterpret_cast<uint8_t *>(pb.out) +
-                      2 * (o_off(pb, b) + h * pb.os_h + (long long)i * pb.os_n);
+                      2 * ((kVarlen ? o_off(pb, b) : b * pb.os_b) + h * pb.os_h + (long long)i * pb.os_n);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -815,7 +824,7 @@ __global__ void __launch_bounds__(128, 1) mma_loop_kernel(int iters, int32_t *si
   }
 }
 
-template <int D, bool SQ, bool FQ>
+template <int D, bool SQ, bool FQ, bool VL>
 cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CUtensorMap &tq,
                                 const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
   using C = Cfg<D>;
@@ -824,14 +833,14 @@ cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CU
   // setmaxnreg.inc could not be satisfied, so such a build is refused.
   static const int launch_regs = [] {
     cudaFuncAttributes fa{};
-    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, SQ, FQ>) == cudaSuccess ? fa.numRegs : -1;
+    return cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, SQ, FQ, VL>) == cudaSuccess ? fa.numRegs : -1;
   }();
   if (launch_regs != int(kLaunchRegs)) return cudaErrorInvalidKernelImage;
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ, FQ>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ, FQ, VL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   const unsigned grid = unsigned(pb.B) * unsigned(pb.Hq) * unsigned(ws.nqb);
-  attn_fwd_kernel<D, SQ, FQ><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
+  attn_fwd_kernel<D, SQ, FQ, VL><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
   return cudaGetLastError();
 }
 
@@ -849,9 +858,13 @@ cudaError_t launch_attention_d(const Problem &pb, const Workspace &ws, const CUt
                                const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream) {
   // Q is fused only without Q smoothing (the smoothed path needs the
   // pre-pass's block means and its Delta S rows)
-  if (pb.smooth_q) return launch_attention_dq<D, true, false>(pb, ws, tq, tk, tv, stream);
-  return pb.q_fused ? launch_attention_dq<D, false, true>(pb, ws, tq, tk, tv, stream)
-                    : launch_attention_dq<D, false, false>(pb, ws, tq, tk, tv, stream);
+  // (variable-length batches are never fused)
+  if (pb.cu_q)
+    return pb.smooth_q ? launch_attention_dq<D, true, false, true>(pb, ws, tq, tk, tv, stream)
+                       : launch_attention_dq<D, false, false, true>(pb, ws, tq, tk, tv, stream);
+  if (pb.smooth_q) return launch_attention_dq<D, true, false, false>(pb, ws, tq, tk, tv, stream);
+  return pb.q_fused ? launch_attention_dq<D, false, true, false>(pb, ws, tq, tk, tv, stream)
+                    : launch_attention_dq<D, false, false, false>(pb, ws, tq, tk, tv, stream);
 }
 
 template <int D>
