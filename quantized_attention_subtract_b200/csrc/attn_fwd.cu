@@ -321,7 +321,7 @@ __device__ __forceinline__ void issue_kv(bool isK, int j, int &n, bool &ok, uint
   if (!ok) return;
   const int st = n % C::kStages;
   const uint32_t ph = (n / C::kStages) & 1;
-  if (!mbar_wait(bars + 8u * uint32_t(kBarEmpty + st), ph ^ 1, status)) {
+  if (!mbar_wait_h(bars + 8u * uint32_t(kBarEmpty + st), ph ^ 1, status)) {
     ok = false;
     return;
   }
@@ -359,7 +359,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // ---- work item: (b, h, query tile); causal runs the longest tiles first
   const int nq = ws.nqb, bhq = pb.B * pb.Hq;
   int qt, bh;
-  if (pb.is_causal) {
+  if (kVarlen) {
+    // only the query tiles inside a sequence are launched
+    int sb, sh;
+    seq_unit(pb.pc_q128, pb.B, pb.Hq, blockIdx.x, sb, sh, qt);
+    bh = sb * pb.Hq + sh;
+  } else if (pb.is_causal) {
     qt = nq - 1 - int(blockIdx.x / bhq);
     bh = int(blockIdx.x % bhq);
   } else {
@@ -477,10 +482,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t dQ = smem_desc_kmajor(sQ, C::Dp);
       int n = 0;
       // with fused Q the INT8 tile was published by the barrier above
-      bool ok = kFuseQ ? true : mbar_wait(bar(kBarQ), 0, status);
+      bool ok = kFuseQ ? true : mbar_wait_h(bar(kBarQ), 0, status);
       auto wait_stage = [&]() -> uint32_t {
         const int st = n % C::kStages;
-        if (ok && !mbar_wait(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
+        if (ok && !mbar_wait_h(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
         return uint32_t(st);
       };
       auto issue_s = [&](uint32_t st) {
@@ -500,13 +505,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
           const uint32_t st = wait_stage();
-          if (ok && !mbar_wait(bar(kBarSEmpty), j & 1, status)) ok = false;
+          if (ok && !mbar_wait_h(bar(kBarSEmpty), j & 1, status)) ok = false;
           if (!ok) break;
           tc_fence_after();
           issue_s(st);
         }
         const uint32_t st = wait_stage();
-        if (ok && !mbar_wait(bar(kBarPFull + (j & 1)), (j >> 1) & 1, status)) ok = false;
+        if (ok && !mbar_wait_h(bar(kBarPFull + (j & 1)), (j >> 1) & 1, status)) ok = false;
         if (!ok) break;
         tc_fence_after();
         const uint64_t dP = smem_desc_kmajor(sP + (j & 1) * C::kPBytes, 128);
@@ -520,7 +525,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       // every MMA issued by this thread has finished before teardown
       mma_commit(bar(kBarFinal));
-      mbar_wait(bar(kBarFinal), 0, status, false);
+      mbar_wait_h(bar(kBarFinal), 0, status, false);
     }
   }
   } else {
@@ -839,7 +844,9 @@ cudaError_t launch_attention_dq(const Problem &pb, const Workspace &ws, const CU
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<D, SQ, FQ, VL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = unsigned(pb.B) * unsigned(pb.Hq) * unsigned(ws.nqb);
+  const unsigned grid = VL ? unsigned(pb.Hq) * unsigned(pb.tot_q128)
+                           : unsigned(pb.B) * unsigned(pb.Hq) * unsigned(ws.nqb);
+  if (grid == 0) return cudaSuccess;
   attn_fwd_kernel<D, SQ, FQ, VL><<<grid, C::kThreads, C::kSmem, stream>>>(tq, tk, tv, pb, ws);
   return cudaGetLastError();
 }

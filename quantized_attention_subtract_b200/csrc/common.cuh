@@ -64,7 +64,36 @@ struct Problem {
   // then the maximum lengths and the batch strides are unused.  Null for
   // the batched layout.  Device copies in the workspace.
   const int *cu_q, *cu_kv;
+  // Variable-length batches only: running totals over the sequences of the
+  // work units that exist -- 128-row query tiles, 64-token and 128-token key
+  // chunks -- (B + 1 entries each, device), and their grand totals, so that
+  // kernels enumerate only units inside a sequence.
+  const int *pc_q128, *pc_kv64, *pc_kv128;
+  int tot_q128, tot_kv64, tot_kv128;
 };
+
+// Sequence b with pc[b] * mul <= x < pc[b + 1] * mul (pc non-decreasing,
+// pc[0] = 0, x < pc[B] * mul): binary search over the B + 1 running totals.
+__device__ __forceinline__ int seq_of(const int *pc, int B, long long mul, long long x) {
+  int lo = 0, hi = B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((long long)pc[mid] * mul <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Unit x of a variable-length enumeration with `heads` heads per sequence:
+// sequence b, head h, unit index t within (b, h) (per-sequence unit counts
+// pc[b + 1] - pc[b]).
+__device__ __forceinline__ void seq_unit(const int *pc, int B, int heads, long long x, int &b, int &h,
+                                         int &t) {
+  b = seq_of(pc, B, heads, x);
+  const int n = pc[b + 1] - pc[b];
+  const long long r = x - (long long)pc[b] * heads;
+  h = int(r / n);
+  t = int(r % n);
+}
 
 // Per batch entry: query / key counts, and the element offset of (token 0,
 // head 0) of q, k, v and out.

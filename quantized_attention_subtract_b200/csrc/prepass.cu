@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
   const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;   // 16 / 21 / 32 row groups
   const int ngroups = blockDim.x / C8;
   const int nchunk = (pb.Nkv + kStatChunk - 1) / kStatChunk;
-  const long long nunits = (long long)pb.B * pb.Hkv * nchunk;
+  // variable-length batches enumerate only the chunks inside a sequence
+  const long long nunits = pb.cu_kv ? (long long)pb.Hkv * pb.tot_kv64 : (long long)pb.B * pb.Hkv * nchunk;
   const long long u0 = nunits * blockIdx.x / gridDim.x, u1 = nunits * (blockIdx.x + 1) / gridDim.x;
   const int stage_bytes = 2 * kStatChunk * rowb;
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm_stats + kStatStages * stage_bytes);
@@ -142,8 +143,15 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
   __syncthreads();
 
   auto unit_src = [&](long long u, int &bh, int &j0, int &n) {
-    bh = int(u / nchunk);
-    j0 = int(u % nchunk) * kStatChunk;
+    if (pb.cu_kv) {
+      int b, h, t;
+      seq_unit(pb.pc_kv64, pb.B, pb.Hkv, u, b, h, t);
+      bh = b * pb.Hkv + h;
+      j0 = t * kStatChunk;
+    } else {
+      bh = int(u / nchunk);
+      j0 = int(u % nchunk) * kStatChunk;
+    }
     n = min(kStatChunk, nkv_of(pb, bh / pb.Hkv) - j0);  // <= 0: past this sequence's end
   };
   auto issue = [&](long long u, int st) {
@@ -369,15 +377,44 @@ struct QUnit {
   long long stride;
 };
 
+// Units of quantize_kernel: K and V tiles (both), then Q blocks unless the
+// attention kernel quantises Q; variable-length batches count only the tiles
+// inside a sequence.
+__host__ __device__ __forceinline__ long long quant_units(const Problem &pb, const Workspace &ws) {
+  const long long nKV = pb.cu_kv ? (long long)pb.Hkv * pb.tot_kv128
+                                 : (long long)pb.B * pb.Hkv * (ws.Nkv_pad / kKVTile);
+  const long long nQ = pb.q_fused ? 0LL : pb.cu_q ? (long long)pb.Hq * pb.tot_q128
+                                                  : (long long)pb.B * pb.Hq * ws.nqb;
+  return 2 * nKV + nQ;
+}
+
+// kVarlen: the unit numbering of a variable-length batch (only the tiles inside
+// a sequence); a template parameter so that the batched kernel, whose thread 0
+// decodes a unit on the path to every unit's barrier, carries none of it.
+// (out of line: the variable-length search would otherwise cost the unit loop
+// registers)
+__device__ __noinline__ int2 seq_unit_ht(const int *pc, int B, int heads, long long x) {
+  int b, h, t;
+  seq_unit(pc, B, heads, x, b, h, t);
+  return make_int2(b * heads + h, t);
+}
+
+template <bool kVarlen>
 __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &ws, long long u) {
   QUnit q{};
   const int nKt = ws.Nkv_pad / kKVTile;
-  const long long nKV = (long long)pb.B * pb.Hkv * nKt;
+  const long long nKV = kVarlen ? (long long)pb.Hkv * pb.tot_kv128 : (long long)pb.B * pb.Hkv * nKt;
   if (u < 2 * nKV) {
     q.kind = int(u & 1);
     const long long kvi = nKV - 1 - (u >> 1);  // reverse head order
-    q.t = int(kvi % nKt);
-    q.bh = int(kvi / nKt);
+    if (kVarlen) {
+      const int2 bt = seq_unit_ht(pb.pc_kv128, pb.B, pb.Hkv, kvi);
+      q.bh = bt.x;
+      q.t = bt.y;
+    } else {
+      q.t = int(kvi % nKt);
+      q.bh = int(kvi / nKt);
+    }
     q.b = q.bh / pb.Hkv;
     q.h = q.bh % pb.Hkv;
     q.r0 = q.t * kKVTile;
@@ -392,8 +429,14 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
   } else {
     const long long qi = u - 2 * nKV;
     q.kind = 2;
-    q.t = int(qi % ws.nqb);
-    q.bh = int(qi / ws.nqb);
+    if (kVarlen) {
+      const int2 bt = seq_unit_ht(pb.pc_q128, pb.B, pb.Hq, qi);
+      q.bh = bt.x;
+      q.t = bt.y;
+    } else {
+      q.t = int(qi % ws.nqb);
+      q.bh = int(qi / ws.nqb);
+    }
     q.b = q.bh / pb.Hq;
     q.h = q.bh % pb.Hq;
     q.r0 = q.t * kQBlk;
@@ -404,6 +447,7 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
   return q;
 }
 
+template <bool kVarlen>
 __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws) {
   extern __shared__ __align__(128) uint8_t sm_q[];
   const int D = pb.D, Dp = ws.Dp, C8 = D / 8, rowb = 2 * D;
@@ -417,9 +461,8 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   unsigned *mslot = reinterpret_cast<unsigned *>(scratch + 66);  // [2 parities][2]
   QUnit *desc = reinterpret_cast<QUnit *>(scratch + 72);    // [stages + 1]
   const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
-  const int nKt = ws.Nkv_pad / kKVTile;
-  // Q blocks come last; they are skipped when the attention kernel quantises Q
-  const long long nunits = 2LL * pb.B * pb.Hkv * nKt + (pb.q_fused ? 0LL : (long long)pb.B * pb.Hq * ws.nqb);
+  // K and V tiles, then Q blocks (skipped when the attention kernel quantises Q)
+  const long long nunits = quant_units(pb, ws);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQuantStages; ++i) mbar_init(b_base + 8 * i, 1);
     fence_mbar_init();
@@ -439,7 +482,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   if (threadIdx.x == 0)
     for (int i = 0; i < kQuantStages; ++i)
       if (blockIdx.x + (long long)i * gridDim.x < nunits)
-        desc[i] = quant_unit(pb, ws, blockIdx.x + (long long)i * gridDim.x);
+        desc[i] = quant_unit<kVarlen>(pb, ws, blockIdx.x + (long long)i * gridDim.x);
   static_assert(kQuantStages + 1 == kSlots, "descriptor ring");
   __syncthreads();
   for (int i = 0; i < kQuantStages; ++i)
@@ -470,7 +513,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
     }
     const long long un = u + (long long)kQuantStages * gridDim.x;
     QUnit *dn = desc + (it + kQuantStages) % kSlots;
-    if (threadIdx.x == 0 && un < nunits) *dn = quant_unit(pb, ws, un);
+    if (threadIdx.x == 0 && un < nunits) *dn = quant_unit<kVarlen>(pb, ws, un);
     __syncthreads();  // stage consumed; next descriptor visible
     if (un < nunits) issue(*dn, st);
 
@@ -676,11 +719,13 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   e = cudaFuncSetAttribute(kv_stats_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)st_smem);
   if (e != cudaSuccess) return e;
   const long long nchunk = (pb.Nkv + kStatChunk - 1) / kStatChunk;
-  const long long su = (long long)pb.B * pb.Hkv * nchunk;
+  const long long su = pb.cu_kv ? (long long)pb.Hkv * pb.tot_kv64 : (long long)pb.B * pb.Hkv * nchunk;
   const unsigned g1 = (unsigned)std::min<long long>(su, 2LL * sms);
-  kv_stats_kernel<<<g1, 256, st_smem, stream>>>(pb, ws);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (g1 > 0) {  // (a variable-length batch may hold no keys at all)
+    kv_stats_kernel<<<g1, 256, st_smem, stream>>>(pb, ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   kv_finalize_kernel<<<pb.B * pb.Hkv, 128, 0, stream>>>(pb, ws);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -688,14 +733,16 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   // stages | output tile | 4 barriers | colsum[128] | chan[128] | scratch[72] | desc[stages + 1]
   const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 72 * 4 +
                         (kQuantStages + 1) * sizeof(QUnit);
-  e = cudaFuncSetAttribute(quantize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
+  auto qk = pb.cu_q ? quantize_kernel<true> : quantize_kernel<false>;
+  e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
   if (e != cudaSuccess) return e;
-  const int nKt = ws.Nkv_pad / kKVTile;
-  const long long nblk = (pb.q_fused ? 0LL : (long long)pb.B * pb.Hq * ws.nqb) + 2LL * pb.B * pb.Hkv * nKt;
+  const long long nblk = quant_units(pb, ws);
   const unsigned g2 = (unsigned)std::min<long long>(nblk, 2LL * sms);
-  quantize_kernel<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (g2 > 0) {
+    qk<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   if (pb.smooth_q) {
     const size_t smem = sizeof(float) * (pb.D * 128 + kDsChunk * pb.D);
     e = cudaFuncSetAttribute(delta_s_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

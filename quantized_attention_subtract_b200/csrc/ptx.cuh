@@ -52,6 +52,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint (the thread may sleep up to the hint, in
+// ns, unless the phase completes first): for the single-thread helper roles
+// (TMA producer, MMA issuer), whose spinning would otherwise take issue slots
+// from the softmax warps of their SM sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_h(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, 20000;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Device-side failure reporting.  `status` is a word in the caller's
 // workspace; a nonzero value makes every other waiter give up quickly.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // one second
@@ -68,6 +84,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int *st
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (honor_abort && *(volatile int *)status != 0) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        atomicCAS(status, 0, kStatusTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// mbar_wait with the hinted try_wait (same limit and abort rules).
+__device__ __forceinline__ bool mbar_wait_h(uint32_t bar, uint32_t parity, int *status,
+                                          bool honor_abort = true) {
+  if (mbar_try_wait_h(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_h(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (honor_abort && *(volatile int *)status != 0) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -104,7 +105,8 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.off_vmin = take(BHk * D * sizeof(unsigned));
   L.off_vinv = take(BHk * D * sizeof(float));
   L.off_status = take(16);
-  L.off_cu = is_varlen(p) ? take(2 * (size_t(p->B) + 1) * sizeof(int32_t)) : 0;
+  // offsets and running unit totals of a variable-length batch: 5 x (B + 1)
+  L.off_cu = is_varlen(p) ? take(5 * (size_t(p->B) + 1) * sizeof(int32_t)) : 0;
   if (p->smooth_q) {
     L.off_mq = take(BHq * L.nqb * D * sizeof(float));
     L.off_dsk = take(BHq * L.nqb * size_t(L.Nkv_pad) * sizeof(float));
@@ -320,14 +322,35 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   Problem pb = make_problem(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (is_varlen(p)) {
-    // the kernels read the (validated) sequence offsets from the workspace
-    int32_t *cu = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(p->workspace) + L.off_cu);
-    const size_t n = (size_t(p->B) + 1) * sizeof(int32_t);
-    if (cudaMemcpyAsync(cu, p->cu_seqlens_q, n, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-        cudaMemcpyAsync(cu + p->B + 1, p->cu_seqlens_kv, n, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    // The kernels read the (validated) sequence offsets from the workspace,
+    // with the running totals of each sequence's query tiles (128 rows) and
+    // key chunks (64 and 128 tokens), so that they enumerate only units
+    // inside a sequence.
+    const int B = p->B;
+    std::vector<int32_t> h(5 * size_t(B + 1), 0);
+    int32_t *cq = h.data(), *ck = cq + B + 1, *pq = ck + B + 1, *p64 = pq + B + 1, *p128 = p64 + B + 1;
+    for (int b = 0; b <= B; ++b) {
+      cq[b] = p->cu_seqlens_q[b];
+      ck[b] = p->cu_seqlens_kv[b];
+    }
+    for (int b = 0; b < B; ++b) {
+      const int lq = cq[b + 1] - cq[b], lk = ck[b + 1] - ck[b];
+      pq[b + 1] = pq[b] + (lq + 127) / 128;
+      p64[b + 1] = p64[b] + (lk + 63) / 64;
+      p128[b + 1] = p128[b] + (lk + 127) / 128;
+    }
+    int32_t *d = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(p->workspace) + L.off_cu);
+    // pageable source: the copy has read h before the call returns
+    if (cudaMemcpyAsync(d, h.data(), h.size() * sizeof(int32_t), cudaMemcpyHostToDevice, st) != cudaSuccess)
       return SAGE_ERR_CUDA;
-    pb.cu_q = cu;
-    pb.cu_kv = cu + p->B + 1;
+    pb.cu_q = d;
+    pb.cu_kv = d + (B + 1);
+    pb.pc_q128 = d + 2 * (B + 1);
+    pb.pc_kv64 = d + 3 * (B + 1);
+    pb.pc_kv128 = d + 4 * (B + 1);
+    pb.tot_q128 = pq[B];
+    pb.tot_kv64 = p64[B];
+    pb.tot_kv128 = p128[B];
   }
   // With fuse_q the whole pass quantises Q inside the attention kernel (it
   // still writes q8 and q_scale to the workspace) and the pre-pass skips Q.
