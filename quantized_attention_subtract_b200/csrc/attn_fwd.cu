@@ -5,8 +5,9 @@
 // ComfyUI blog, part 2; "sageattention" package page, "What it is"):
 //   S = q8 k8^T                    exact int32, tensor cores (kind::i8)
 //   s = S * q_scale * k_scale * sm_scale * log2(e)   (+ dS for smoothed Q)
-//   online softmax in base 2 with running max m and sum l
-//   P8 = e4m3(448 * 2^(s - m))     FP8 probabilities
+//   online softmax in base 2 with a lazily raised reference max m (raised
+//   only past m + 1) and sum l
+//   P8 = e4m3(224 * 2^(s - m))     FP8 probabilities (<= 448 since s <= m + 1)
 //   O += P8 v8                     fp32 accumulation, tensor cores (kind::f8f6f4)
 //   out = O * v_scale / l (+ mean_v), rounded to bf16 / fp16
 //
@@ -19,6 +20,7 @@
 //   warp 1      allocates 256 TMEM columns; lane 0 issues the MMAs:
 //               S_{j+1} = Q K_{j+1}^T as soon as softmax has read S_j, then
 //               O += P_j V_j once P_j is in shared memory
+//               (both single-thread roles wait with a suspend-time hint)
 //   warps 2-3   idle
 //   warps 4-7   softmax: one query row per thread (TMEM lane), reads S with
 //               tcgen05.ld, writes P_j (swizzled, double-buffered) to shared
@@ -28,6 +30,11 @@
 // TMEM: S at columns [0,128), O at [128, 128 + D).
 // Causal tiles past the diagonal are skipped; keys >= Nkv and (causal)
 // keys > query are masked; rows >= Nq are computed but not stored.
+// Template flags: smoothed Q (dS added to the logits), fused Q (the CTA
+// quantises its own Q tile from the 16-bit input before the roles split),
+// variable-length batches (per-sequence lengths and offsets; only query tiles
+// inside a sequence are launched).
+// Every tcgen05.ld / st here runs under warp-uniform control flow (.sync.aligned).
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>

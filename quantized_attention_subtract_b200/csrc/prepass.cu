@@ -7,21 +7,26 @@
 // block to INT8 and V to FP8 (closerAI ComfyUI blog, part 2).
 //
 // Four kernels on one stream:
-//   kv_stats   per (b, kv head, 256-token chunk): fixed-point channel sums of
-//              K (and V) and the V channel max/min, combined with atomics
-//              (integer addition is exact, so the order does not matter);
+//   kv_stats   persistent; contiguous runs of (b, kv head, 64-token chunk)
+//              units per CTA: fixed-point channel sums of K (and V) and the V
+//              channel max/min in registers, flushed with atomics when the run
+//              changes head (integer addition is exact, so the order does not
+//              matter);
 //   kv_finalize per (b, kv head): mean_k, mean_v, V channel scale and its
 //              reciprocal, once per channel;
-//   quantize   per 128-token tile of K, V or Q (in that order, K/V heads in
+//   quantize   persistent over 128-token tiles of K, V, then Q (K/V heads in
 //              reverse so their second read hits L2): smoothing, block amax,
-//              INT8/FP8 codes written through shared memory as whole
-//              coalesced tiles in the attention kernel's layout (V
-//              transposed so that keys are contiguous);
+//              INT8 codes of K and Q stored from registers, FP8 codes of V
+//              transposed through shared memory (keys contiguous), all in the
+//              attention kernel's layout;
 //   delta_s    (smooth_q only) the correction dS[blk][j] = mq[blk] . K'_j,
 //              stored pre-multiplied by sm_scale * log2(e).
 //
 // Threads own 16-byte chunks (8 channels) of rows, so loads are 16-byte
-// vectors and a warp covers whole rows.
+// vectors and a warp covers whole rows.  Rows arrive in shared memory through
+// cp.async.bulk copies on an mbarrier ring: one copy per unit when tokens are
+// dense, one per row otherwise.  Variable-length batches enumerate only the
+// units inside a sequence.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
