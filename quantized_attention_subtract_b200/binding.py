@@ -273,8 +273,13 @@ _HOST_CHUNK_MIN_BYTES = 8 << 20
 _HOST_MAX_CHUNKS = 16
 
 
-def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int):
-    """Split (batch, kv head) into contiguous slices [(b, h0, h1)] of whole kv heads."""
+def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int, layout: str = "HND"):
+    """Split (batch, kv head) into slices [(b, h0, h1)] of whole kv heads that
+    are contiguous in host memory: head ranges of one batch entry for HND, whole
+    batch entries for NHD (a head range of an NHD tensor is strided, and a
+    strided host-to-device copy goes through a pageable staging copy)."""
+    if layout == "NHD":
+        return [(b, 0, Hkv) for b in range(B)]
     total = B * Hkv
     n = max(1, min(_HOST_MAX_CHUNKS, total, (total * bytes_per_kv_head) // _HOST_CHUNK_MIN_BYTES))
     per_batch = -(-n // B)                       # chunks per batch entry
@@ -298,7 +303,7 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
     qd, kd, vd = (torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (q, k, v))
     od = torch.empty(q.shape, dtype=q.dtype, device=dev)
     per_kv = (k.element_size() * Nkv * D * 2 + q.element_size() * group * Nq * D * 2)
-    chunks = _host_chunks(B, Hkv, group, per_kv)
+    chunks = _host_chunks(B, Hkv, group, per_kv, layout)
 
     def sl(t, b, h0, h1):
         idx = [slice(b, b + 1), slice(None), slice(None), slice(None)]

@@ -70,6 +70,20 @@ struct Problem {
   // kernels enumerate only units inside a sequence.
   const int *pc_q128, *pc_kv64, *pc_kv128;
   int tot_q128, tot_kv64, tot_kv128;
+  // Pre-pass loads of inputs whose tokens are strided (NHD, packed
+  // variable-length batches, padded rows): 1 when the pre-pass reads that
+  // tensor through the tensor maps of InputMaps (one box per unit) instead of
+  // one bulk copy per row; *_hn: map dimension order (D, H, N, B) instead of
+  // (D, N, H, B).  A variable-length batch's map spans all packed tokens with
+  // a batch extent of 1.
+  int k_map, v_map, q_map;
+  int k_hn, v_hn, q_hn;
+};
+
+// Tensor maps of the caller's 16-bit inputs for the pre-pass: boxes of D
+// channels x 64 tokens (kv_stats) and x 128 tokens (quantize) of one head.
+struct InputMaps {
+  CUtensorMap k64, v64, k128, v128, q128;
 };
 
 // Sequence b with pc[b] * mul <= x < pc[b + 1] * mul (pc non-decreasing,
@@ -132,7 +146,8 @@ __device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c,
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t stream);
+cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMaps &im,
+                           cudaStream_t stream);
 cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
                              const CUtensorMap &tm_k, const CUtensorMap &tm_v, cudaStream_t stream);
 cudaError_t launch_dump_s(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,

@@ -24,9 +24,11 @@
 //
 // Threads own 16-byte chunks (8 channels) of rows, so loads are 16-byte
 // vectors and a warp covers whole rows.  Rows arrive in shared memory through
-// cp.async.bulk copies on an mbarrier ring: one copy per unit when tokens are
-// dense, one per row otherwise.  Variable-length batches enumerate only the
-// units inside a sequence.
+// copies on an mbarrier ring: one cp.async.bulk per unit when tokens are
+// dense, one tensor-map box per unit when they are strided (NHD, packed
+// variable-length batches, padded rows; one bulk copy per row if the driver
+// rejects the map).  Variable-length batches enumerate only the units inside
+// a sequence.
 #include <algorithm>
 #include <cstdint>
 #include <cuda_runtime.h>
@@ -114,6 +116,35 @@ __device__ __forceinline__ void issue_rows(uint32_t dst, const uint16_t *src, lo
   }
 }
 
+// Tensor-map load of one box (D channels x the map's token count) of head h
+// of batch entry b, from token r0 of that entry on: a variable-length batch's
+// map spans all packed tokens (entry b starts at token cu[b]) with a batch
+// extent of 1.  x = 0, so the 16-byte rule on the innermost coordinate holds.
+__device__ __forceinline__ void map_load(uint32_t dst, const CUtensorMap *m, uint32_t bar, int hn,
+                                         const int *cu, int b, int h, int r0) {
+  const int tok = (cu ? cu[b] : 0) + r0, bb = cu ? 0 : b;
+  if (hn) tma_load_4d(dst, m, bar, 0, h, tok, bb);
+  else tma_load_4d(dst, m, bar, 0, tok, h, bb);
+}
+
+// Thread 0 of a block: arm `bar` with `bytes` and load one box (out of line,
+// so that the unit loop that calls it keeps its registers).
+__device__ __noinline__ void map_issue(uint32_t dst, const CUtensorMap *m, uint32_t bar, uint32_t bytes,
+                                       int hn, const int *cu, int b, int h, int r0) {
+  mbar_arrive_expect_tx(bar, bytes);
+  map_load(dst, m, bar, hn, cu, b, h, r0);
+}
+
+// Tensor-map boxes land at 128-byte aligned shared addresses: the dynamic
+// shared array is declared 1024-byte aligned, and a block whose base is not
+// 128-byte aligned reports SAGE_ERR_ALIGNMENT and does nothing (block-uniform,
+// before any barrier exists).
+__device__ __forceinline__ bool smem_misaligned(const uint8_t *base, int *status) {
+  if ((smem_u32(base) & 127u) == 0) return false;
+  if (threadIdx.x == 0) atomicCAS(status, 0, kStatusAlignment);
+  return true;
+}
+
 // Block-wide bounded wait; every thread learns whether it succeeded.
 __device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity, int *status) {
   const bool ok = mbar_wait(bar, parity, status);
@@ -128,8 +159,11 @@ __device__ __forceinline__ bool block_wait(uint32_t bar, uint32_t parity, int *s
 // Stage: 64 K rows then 64 V rows (K only when smooth_k).
 constexpr int kStatStages = 2;
 
-__global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace ws) {
-  extern __shared__ __align__(128) uint8_t sm_stats[];
+__global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace ws,
+                                                          const __grid_constant__ CUtensorMap mk,
+                                                          const __grid_constant__ CUtensorMap mv) {
+  extern __shared__ __align__(1024) uint8_t sm_stats[];
+  if (smem_misaligned(sm_stats, ws.status)) return;
   const int D = pb.D, C8 = D / 8, rowb = 2 * D;
   const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;   // 16 / 21 / 32 row groups
   const int ngroups = blockDim.x / C8;
@@ -169,18 +203,25 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
       if (threadIdx.x == 0) mbar_arrive(bar);
       return;
     }
-    const uint32_t bytes = uint32_t(n) * rowb * (pb.smooth_k ? 2 : 1);
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, bytes);
+    // a tensor-map box always lands whole (rows past the tensor read as zero)
+    const uint32_t kbytes = pb.smooth_k ? uint32_t(pb.k_map ? kStatChunk : n) * rowb : 0u;
+    const uint32_t vbytes = uint32_t(pb.v_map ? kStatChunk : n) * rowb;
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(bar, kbytes + vbytes);
     const uint16_t *ksrc = pb.k + k_off(pb, b) + h * pb.ks_h + j0 * pb.ks_n;
     const uint16_t *vsrc = pb.v + v_off(pb, b) + h * pb.vs_h + j0 * pb.vs_n;
-    // dense tokens: one copy per tensor; otherwise one per row (K rows by
-    // threads 0.., V rows by threads ..127)
-    if (pb.ks_n == D) {
+    // strided tokens with a tensor map: one box per tensor; dense tokens: one
+    // copy per tensor; otherwise one per row (K rows by threads 0.., V rows by
+    // threads ..127)
+    if (pb.k_map) {
+      if (pb.smooth_k && threadIdx.x == 0) map_load(dst, &mk, bar, pb.k_hn, pb.cu_kv, b, h, j0);
+    } else if (pb.ks_n == D) {
       if (pb.smooth_k && threadIdx.x == 0) bulk_load(dst, ksrc, uint32_t(n) * rowb, bar);
     } else if (pb.smooth_k && int(threadIdx.x) < n) {
       bulk_load(dst + threadIdx.x * rowb, ksrc + threadIdx.x * pb.ks_n, rowb, bar);
     }
-    if (pb.vs_n == D) {
+    if (pb.v_map) {
+      if (threadIdx.x == 32) map_load(dst + kStatChunk * rowb, &mv, bar, pb.v_hn, pb.cu_kv, b, h, j0);
+    } else if (pb.vs_n == D) {
       if (threadIdx.x == 127) bulk_load(dst + kStatChunk * rowb, vsrc, uint32_t(n) * rowb, bar);
     } else if (int(threadIdx.x) >= 128 - n && threadIdx.x < 128) {
       const int r = threadIdx.x - (128 - n);
@@ -452,9 +493,15 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
   return q;
 }
 
-template <bool kVarlen>
-__global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws) {
-  extern __shared__ __align__(128) uint8_t sm_q[];
+// kMaps: some input is read through a tensor map (a template parameter, so
+// that the kernel for dense inputs carries none of it).
+template <bool kVarlen, bool kMaps>
+__global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace ws,
+                                                          const __grid_constant__ CUtensorMap mk,
+                                                          const __grid_constant__ CUtensorMap mv,
+                                                          const __grid_constant__ CUtensorMap mq) {
+  extern __shared__ __align__(1024) uint8_t sm_q[];
+  if (smem_misaligned(sm_q, ws.status)) return;
   const int D = pb.D, Dp = ws.Dp, C8 = D / 8, rowb = 2 * D;
   const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;  // rows 4 rg .. 4 rg + 3
   const int stage_bytes = 128 * rowb;
@@ -481,6 +528,18 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
   // barrier.
   constexpr int kSlots = kQuantStages + 1;
   auto issue = [&](const QUnit &q, int st) {
+    if constexpr (kMaps) {
+      const int use_map = q.kind == 0 ? pb.k_map : q.kind == 1 ? pb.v_map : pb.q_map;
+      if (use_map) {
+        // one box of 128 tokens (rows past nvalid are loaded but never used)
+        if (threadIdx.x == 0)
+          map_issue(s_base + st * stage_bytes, q.kind == 0 ? &mk : q.kind == 1 ? &mv : &mq,
+                    b_base + 8 * st, uint32_t(stage_bytes),
+                    q.kind == 0 ? pb.k_hn : q.kind == 1 ? pb.v_hn : pb.q_hn,
+                    q.kind == 2 ? pb.cu_q : pb.cu_kv, q.b, q.h, q.r0);
+        return;
+      }
+    }
     issue_rows(s_base + st * stage_bytes, q.src, q.stride, q.nvalid, rowb, b_base + 8 * st, true,
                uint32_t(q.nvalid) * rowb);
   };
@@ -706,7 +765,8 @@ __global__ void __launch_bounds__(128) delta_s_kernel(Problem pb, Workspace ws) 
 
 }  // namespace
 
-cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t stream) {
+cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMaps &im,
+                           cudaStream_t stream) {
   const long long nch = (long long)pb.B * pb.Hkv * pb.D;
   // sums (int64) and max keys start at zero; min keys at all-ones
   cudaError_t e = cudaMemsetAsync(ws.k_sum, 0, nch * (2 * sizeof(long long) + sizeof(unsigned)),
@@ -727,7 +787,7 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   const long long su = pb.cu_kv ? (long long)pb.Hkv * pb.tot_kv64 : (long long)pb.B * pb.Hkv * nchunk;
   const unsigned g1 = (unsigned)std::min<long long>(su, 2LL * sms);
   if (g1 > 0) {  // (a variable-length batch may hold no keys at all)
-    kv_stats_kernel<<<g1, 256, st_smem, stream>>>(pb, ws);
+    kv_stats_kernel<<<g1, 256, st_smem, stream>>>(pb, ws, im.k64, im.v64);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -738,13 +798,15 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, cudaStream_t 
   // stages | output tile | 4 barriers | colsum[128] | chan[128] | scratch[72] | desc[stages + 1]
   const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 72 * 4 +
                         (kQuantStages + 1) * sizeof(QUnit);
-  auto qk = pb.cu_q ? quantize_kernel<true> : quantize_kernel<false>;
+  const bool maps = pb.k_map || pb.v_map || pb.q_map;
+  auto qk = pb.cu_q ? (maps ? quantize_kernel<true, true> : quantize_kernel<true, false>)
+                    : (maps ? quantize_kernel<false, true> : quantize_kernel<false, false>);
   e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)q_smem);
   if (e != cudaSuccess) return e;
   const long long nblk = quant_units(pb, ws);
   const unsigned g2 = (unsigned)std::min<long long>(nblk, 2LL * sms);
   if (g2 > 0) {
-    qk<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws);
+    qk<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws, im.k128, im.v128, im.q128);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

@@ -72,6 +72,7 @@ __device__ __forceinline__ bool mbar_try_wait_h(uint32_t bar, uint32_t parity) {
 // workspace; a nonzero value makes every other waiter give up quickly.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // one second
 constexpr int kStatusTimeout = 5;                                 // SAGE_ERR_DEVICE_TIMEOUT
+constexpr int kStatusAlignment = 3;                               // SAGE_ERR_ALIGNMENT
 
 // Wait for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording a timeout) when one second passes first.  With

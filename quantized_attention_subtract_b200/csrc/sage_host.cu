@@ -280,6 +280,64 @@ bool make_q_input_map(const Problem &pb, CUtensorMap *m, int *hn) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tensor map of a caller's 16-bit input (element strides s_b, s_h, s_n; the
+// channel stride is 1) for the pre-pass: dimensions (D, N, H, B), or
+// (D, H, N, B) when the head stride is the smaller one, so the strides
+// increase; box D channels x `rows` tokens of one head, no swizzle, zero fill
+// past N.  A variable-length batch passes the packed token count as N and
+// B = 1.  Returns false when the driver rejects the map (the pre-pass then
+// copies rows one by one).
+bool make_input_map(const uint16_t *base, int bf16, int D, long long s_b, long long s_h,
+                    long long s_n, long long H, long long N, long long B, uint32_t rows,
+                    CUtensorMap *m, int *hn) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || N <= 0 || H <= 0 || B <= 0) return false;
+  const bool head_inner = s_h < s_n;
+  *hn = head_inner ? 1 : 0;
+  const long long sb = B == 1 ? (head_inner ? N * s_n : H * s_h) : s_b;
+  const cuuint64_t dims[4] = {cuuint64_t(D), cuuint64_t(head_inner ? H : N),
+                              cuuint64_t(head_inner ? N : H), cuuint64_t(B)};
+  const cuuint64_t strides[3] = {cuuint64_t(2 * (head_inner ? s_h : s_n)),
+                                 cuuint64_t(2 * (head_inner ? s_n : s_h)), cuuint64_t(2 * sb)};
+  const cuuint32_t box[4] = {cuuint32_t(D), head_inner ? 1u : rows, head_inner ? rows : 1u, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+            const_cast<uint16_t *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Input maps for every input the pre-pass reads whose tokens are not dense
+// (token stride != D); dense inputs keep one bulk copy per unit.  nq_tot /
+// nkv_tot: packed token counts of a variable-length batch (0 otherwise).
+void make_input_maps(Problem &pb, InputMaps &im, long long nq_tot, long long nkv_tot) {
+  const bool vl = pb.cu_q != nullptr;
+  const long long Bm = vl ? 1 : pb.B;
+  const long long Nk = vl ? nkv_tot : pb.Nkv, Nq = vl ? nq_tot : pb.Nq;
+  int hn0 = 0, hn1 = 0;
+  if (pb.ks_n != pb.D && pb.smooth_k &&
+      make_input_map(pb.k, pb.bf16, pb.D, pb.ks_b, pb.ks_h, pb.ks_n, pb.Hkv, Nk, Bm, 64, &im.k64, &hn0) &&
+      make_input_map(pb.k, pb.bf16, pb.D, pb.ks_b, pb.ks_h, pb.ks_n, pb.Hkv, Nk, Bm, 128, &im.k128, &hn1)) {
+    pb.k_map = 1;
+    pb.k_hn = hn0;
+  } else if (pb.ks_n != pb.D && !pb.smooth_k &&
+             make_input_map(pb.k, pb.bf16, pb.D, pb.ks_b, pb.ks_h, pb.ks_n, pb.Hkv, Nk, Bm, 128, &im.k128, &hn1)) {
+    pb.k_map = 1;  // kv_stats does not read K without smooth_k
+    pb.k_hn = hn1;
+  }
+  if (pb.vs_n != pb.D &&
+      make_input_map(pb.v, pb.bf16, pb.D, pb.vs_b, pb.vs_h, pb.vs_n, pb.Hkv, Nk, Bm, 64, &im.v64, &hn0) &&
+      make_input_map(pb.v, pb.bf16, pb.D, pb.vs_b, pb.vs_h, pb.vs_n, pb.Hkv, Nk, Bm, 128, &im.v128, &hn1)) {
+    pb.v_map = 1;
+    pb.v_hn = hn0;
+  }
+  if (pb.qs_n != pb.D && !pb.q_fused &&
+      make_input_map(pb.q, pb.bf16, pb.D, pb.qs_b, pb.qs_h, pb.qs_n, pb.Hq, Nq, Bm, 128, &im.q128, &hn0)) {
+    pb.q_map = 1;
+    pb.q_hn = hn0;
+  }
+}
+
 bool make_maps(const sage_attn_params_t *p, const Workspace &ws, Maps &m) {
   const uint64_t BHq = uint64_t(p->B) * p->Hq, BHk = uint64_t(p->B) * p->Hkv;
   return make_map(&m.q, ws.q8, ws.Dp, BHq * ws.Nq_pad, ws.Dp, 128) &&
@@ -321,6 +379,7 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   const Workspace ws = make_workspace(p, L);
   Problem pb = make_problem(p);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  long long nq_tot = 0, nkv_tot = 0;  // packed token counts (variable-length batches)
   if (is_varlen(p)) {
     // The kernels read the (validated) sequence offsets from the workspace,
     // with the running totals of each sequence's query tiles (128 rows) and
@@ -351,6 +410,8 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
     pb.tot_q128 = pq[B];
     pb.tot_kv64 = p64[B];
     pb.tot_kv128 = p128[B];
+    nq_tot = cq[B];
+    nkv_tot = ck[B];
   }
   // With fuse_q the whole pass quantises Q inside the attention kernel (it
   // still writes q8 and q_scale to the workspace) and the pre-pass skips Q.
@@ -364,7 +425,12 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
     }
   }
   if (pre && cudaMemsetAsync(ws.status, 0, sizeof(int), st) != cudaSuccess) return SAGE_ERR_CUDA;
-  if (pre && launch_prepass(pb, ws, st) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (pre) {
+    InputMaps im;
+    std::memset(&im, 0, sizeof(im));
+    make_input_maps(pb, im, nq_tot, nkv_tot);
+    if (launch_prepass(pb, ws, im, st) != cudaSuccess) return SAGE_ERR_CUDA;
+  }
   if (attn) {
     CUtensorMap q_input = m.q;
     if (!make_maps(p, ws, m)) return SAGE_ERR_CUDA;

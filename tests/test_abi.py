@@ -191,3 +191,27 @@ def test_varlen_workspace_holds_the_offsets():
     _, n0 = _ws_size(batched)
     _, n1 = _ws_size(_varlen_params([0, 100, 256], [0, 200, 256]))
     assert n1 > n0
+
+
+@pytest.mark.parametrize("layout,B,Hkv,group,N", [("HND", 4, 32, 1, 4096), ("HND", 1, 8, 4, 32768),
+                                                   ("HND", 2, 3, 2, 64), ("NHD", 2, 48, 1, 17776),
+                                                   ("NHD", 1, 4, 4, 100)])
+def test_host_chunks_cover_every_head_once_in_contiguous_slices(layout, B, Hkv, group, N):
+    """Host-tensor calls are pipelined over chunks of whole kv heads; every
+    (batch, kv head) is in exactly one chunk, and each chunk's slice of a
+    dense host tensor is contiguous (a strided slice would be copied through
+    pageable staging memory)."""
+    import torch
+    D = 64
+    per_kv = 2 * N * D * 2 + 2 * group * N * D * 2
+    chunks = binding._host_chunks(B, Hkv, group, per_kv, layout)
+    seen = [(b, h) for b, h0, h1 in chunks for h in range(h0, h1)]
+    assert sorted(seen) == [(b, h) for b in range(B) for h in range(Hkv)]
+    shape = (B, Hkv * group, N, D) if layout == "HND" else (B, N, Hkv * group, D)
+    q = torch.empty(shape, dtype=torch.float16)
+    for b, h0, h1 in chunks:
+        if layout == "HND":
+            view = q[b:b + 1, h0 * group:h1 * group]
+        else:
+            view = q[b:b + 1, :, h0 * group:h1 * group]
+        assert view.is_contiguous(), (b, h0, h1)

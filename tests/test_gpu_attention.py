@@ -83,6 +83,18 @@ def test_public_api_matches_params_path_and_host_tensors():
     assert torch.equal(h, g.out.cpu())
 
 
+def test_host_tensors_nhd():
+    """Host tensors in NHD layout (copied one whole batch entry at a time) give
+    the device path's output bit for bit."""
+    w = random_problem(2, 4, 2, 300, 260, 64, layout="NHD", dtype="fp16", seed=6)
+    q, k, v = generate(w)
+    g = GpuRun(w, q, k, v)
+    h = sageattn(g.q.cpu().pin_memory(), g.k.cpu().pin_memory(), g.v.cpu().pin_memory(),
+                 tensor_layout="NHD")
+    torch.cuda.synchronize()
+    assert torch.equal(h, g.out.cpu())
+
+
 def test_strided_inputs():
     """q, k, v as views with padded token strides (still 16-byte aligned rows)."""
     w = random_problem(1, 2, 2, 256, 256, 64, dtype="fp16", seed=5)
