@@ -92,6 +92,12 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, int *st
   const bool ok = mbar_wait(bar, parity, status);
   return __all_sync(0xffffffffu, ok);
 }
+// The same with the suspend-time hint (the single-issuer roles' waits).
+__device__ __forceinline__ bool warp_wait_h(uint32_t bar, uint32_t parity, int *status,
+                                            bool honor_abort = true) {
+  const bool ok = mbar_wait_h(bar, parity, status, honor_abort);
+  return __all_sync(0xffffffffu, ok);
+}
 
 // One query row's share of one KV tile (128 keys), in two parts around the
 // lazy reference-max update.
@@ -343,6 +349,36 @@ __device__ __forceinline__ void issue_kv(bool isK, int j, int &n, bool &ok, uint
   ++n;
 }
 
+// The same issued by a whole warp (warp-uniform control flow, so that the
+// coordinates stay in uniform registers): every lane waits for the stage,
+// the elected lane arms its barrier and issues the copy.
+template <int D>
+__device__ __forceinline__ void issue_kv_warp(bool isK, int j, int &n, bool &ok, bool leader,
+                                              uint32_t bars, uint32_t sRing, const CUtensorMap *tm_k,
+                                              const CUtensorMap *tm_v, int krow0, int vrow0,
+                                              int *status) {
+  using C = Cfg<D>;
+  if (!ok) return;
+  const int st = n % C::kStages;
+  const uint32_t ph = (n / C::kStages) & 1;
+  if (!warp_wait_h(bars + 8u * uint32_t(kBarEmpty + st), ph ^ 1, status)) {
+    ok = false;
+    return;
+  }
+  const uint32_t dst = sRing + st * C::kStageBytes, full = bars + 8u * uint32_t(kBarFull + st);
+  if (leader) {
+    if (isK) {
+      mbar_arrive_expect_tx(full, C::kKBytes);
+      tma_load_2d(dst, tm_k, full, 0, krow0 + j * kKVTile);
+    } else {
+      mbar_arrive_expect_tx(full, C::kVBytes);
+      tma_load_2d(dst, tm_v, full, j * kKVTile, vrow0);
+    }
+  }
+  __syncwarp();
+  ++n;
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -452,23 +488,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   reg_dealloc<kHelperRegs>();
   if (warp == 0) {
     // ================================================= TMA producer
-    if (lane == 0 && !skip_all) {
+    // The whole warp runs the loop; the elected lane issues the copies.
+    if (!skip_all) {
+      const bool leader = elect_one();
       if constexpr (!kFuseQ) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-        mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
-        tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+        if (leader) {
+          tma_prefetch_desc(&tm_q);
+          tma_prefetch_desc(&tm_k);
+          tma_prefetch_desc(&tm_v);
+          mbar_arrive_expect_tx(bar(kBarQ), C::kQBytes);
+          tma_load_2d(sQ, &tm_q, bar(kBarQ), 0, bh * ws.Nq_pad + q0);
+        }
+        __syncwarp();
       }
-      int n = n_carry;
+      // (thread 0 issued the first n_carry loads before the roles split)
+      const int carried = kFuseQ ? __shfl_sync(0xffffffffu, n_carry, 0) : 0;
+      int n = carried;
       bool ok = true;
-      // K_0, K_1, V_0, K_2, V_1, ... skipping the n_carry loads issued early
+      // K_0, K_1, V_0, K_2, V_1, ... skipping the loads issued early
       int pos = 0;
       auto issue = [&](bool isK, int j) {
         if constexpr (kFuseQ) {
-          if (pos++ < n_carry) return;
+          if (pos++ < carried) return;
         }
-        issue_kv<D>(isK, j, n, ok, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D, status);
+        issue_kv_warp<D>(isK, j, n, ok, leader, bars, sRing, &tm_k, &tm_v, bhk * ws.Nkv_pad, bhk * D,
+                         status);
       };
       issue(true, 0);
       for (int j = 0; j < T; ++j) {
@@ -476,32 +520,44 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         issue(false, j);
       }
       // Before leaving, make sure every copy issued has landed (bounded).
-      mbar_wait(bar(kBarQ), 0, status, false);
+      warp_wait_h(bar(kBarQ), 0, status, false);
       for (int m = (n > C::kStages ? n - C::kStages : 0); m < n; ++m)
-        mbar_wait(bar(kBarFull + m % C::kStages), (m / C::kStages) & 1, status, false);
+        warp_wait_h(bar(kBarFull + m % C::kStages), (m / C::kStages) & 1, status, false);
     }
   } else if (warp == 1) {
     // ================================================= MMA issuer
-    if (lane == 0 && !skip_all) {
+    // The whole warp runs the loop (warp-uniform control flow, so that the
+    // descriptors stay in uniform registers); the elected lane issues the
+    // MMAs and commits.  Descriptors of the ring stages and P buffers differ
+    // only in their start-address field (16-byte units, bits [0, 14)).
+    if (!skip_all) {
+      const bool leader = elect_one();
       const uint32_t tS = tmem, tO = tmem + 128;
-      const uint32_t id_s = idesc_i8(128, 128);
-      const uint32_t id_o = idesc_e4m3_f32(128, D);
+      constexpr uint32_t id_s = idesc_i8(128, 128);
+      constexpr uint32_t id_o = idesc_e4m3_f32(128, D);
+      constexpr uint64_t kStageStep = uint64_t(C::kStageBytes) >> 4, kPStep = uint64_t(C::kPBytes) >> 4;
       const uint64_t dQ = smem_desc_kmajor(sQ, C::Dp);
+      const uint64_t dK0 = smem_desc_kmajor(sRing, C::Dp);
+      const uint64_t dV0 = smem_desc_kmajor(sRing, 128);
+      const uint64_t dP0 = smem_desc_kmajor(sP, 128);
       int n = 0;
       // with fused Q the INT8 tile was published by the barrier above
-      bool ok = kFuseQ ? true : mbar_wait_h(bar(kBarQ), 0, status);
+      bool ok = kFuseQ ? true : warp_wait_h(bar(kBarQ), 0, status);
       auto wait_stage = [&]() -> uint32_t {
         const int st = n % C::kStages;
-        if (ok && !mbar_wait_h(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
+        if (ok && !warp_wait_h(bar(kBarFull + st), (n / C::kStages) & 1, status)) ok = false;
         return uint32_t(st);
       };
       auto issue_s = [&](uint32_t st) {
-        const uint64_t dK = smem_desc_kmajor(sRing + st * C::kStageBytes, C::Dp);
+        const uint64_t dK = dK0 + st * kStageStep;
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < C::kQKSteps; ++k)
-          mma_i8_ss(tS, dQ + 2 * k, dK + 2 * k, id_s, k > 0 ? 1u : 0u);
-        mma_commit(bar(kBarSFull));
-        mma_commit(bar(kBarEmpty + st));
+          for (int k = 0; k < C::kQKSteps; ++k)
+            mma_i8_ss(tS, dQ + 2 * k, dK + 2 * k, id_s, k > 0 ? 1u : 0u);
+          mma_commit(bar(kBarSFull));
+          mma_commit(bar(kBarEmpty + st));
+        }
+        __syncwarp();
         ++n;
       };
       if (ok) {
@@ -512,27 +568,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       for (int j = 0; ok && j < T; ++j) {
         if (j + 1 < T) {
           const uint32_t st = wait_stage();
-          if (ok && !mbar_wait_h(bar(kBarSEmpty), j & 1, status)) ok = false;
+          if (ok && !warp_wait_h(bar(kBarSEmpty), j & 1, status)) ok = false;
           if (!ok) break;
           tc_fence_after();
           issue_s(st);
         }
         const uint32_t st = wait_stage();
-        if (ok && !mbar_wait_h(bar(kBarPFull + (j & 1)), (j >> 1) & 1, status)) ok = false;
+        if (ok && !warp_wait_h(bar(kBarPFull + (j & 1)), (j >> 1) & 1, status)) ok = false;
         if (!ok) break;
         tc_fence_after();
-        const uint64_t dP = smem_desc_kmajor(sP + (j & 1) * C::kPBytes, 128);
-        const uint64_t dV = smem_desc_kmajor(sRing + st * C::kStageBytes, 128);
+        const uint64_t dP = dP0 + uint64_t(j & 1) * kPStep;
+        const uint64_t dV = dV0 + st * kStageStep;
+        if (leader) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_f8_ss(tO, dP + 2 * k, dV + 2 * k, id_o, (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(bar(kBarPVDone + (j & 1)));
-        mma_commit(bar(kBarEmpty + st));
+          for (int k = 0; k < 4; ++k)
+            mma_f8_ss(tO, dP + 2 * k, dV + 2 * k, id_o, (j > 0 || k > 0) ? 1u : 0u);
+          mma_commit(bar(kBarPVDone + (j & 1)));
+          mma_commit(bar(kBarEmpty + st));
+        }
+        __syncwarp();
         ++n;
       }
-      // every MMA issued by this thread has finished before teardown
-      mma_commit(bar(kBarFinal));
-      mbar_wait_h(bar(kBarFinal), 0, status, false);
+      // every MMA issued by the elected lane has finished before teardown
+      if (leader) mma_commit(bar(kBarFinal));
+      __syncwarp();
+      warp_wait_h(bar(kBarFinal), 0, status, false);
     }
   }
   } else {

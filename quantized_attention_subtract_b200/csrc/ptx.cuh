@@ -363,6 +363,17 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// One lane of the (converged) warp gets true: elect.sync over all 32 lanes.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t leader;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(leader));
+  return leader != 0;
+}
+
 // max of three floats in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
