@@ -28,6 +28,10 @@ CASES = [
     dict(args=(1, 8, 1, 129, 1100, 128), dtype="bf16"),                     # GQA 8:1, ragged
     dict(args=(1, 2, 2, 1, 1, 64), dtype="fp16"),                           # one query, one key
     dict(args=(1, 2, 1, 5, 3000, 96), dtype="fp16", smooth_v=True),
+    # NHD without smooth_k (the pre-pass reads K only for quantisation) and
+    # NHD with smoothed Q and V, both through the pre-pass's tensor maps
+    dict(args=(2, 4, 2, 200, 333, 128), dtype="bf16", layout="NHD", smooth_k=False),
+    dict(args=(1, 4, 4, 260, 390, 96), dtype="fp16", layout="NHD", smooth_q=True, smooth_v=True),
 ]
 
 
