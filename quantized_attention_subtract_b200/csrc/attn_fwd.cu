@@ -17,10 +17,11 @@
 // (setmaxnreg).
 //   warp 0      TMA producer: Q once, then K_0, K_1, V_0, K_2, V_1, ... into a
 //               3-stage shared-memory ring (order = MMA consumption order)
-//   warp 1      allocates 256 TMEM columns; lane 0 issues the MMAs:
+//   warp 1      allocates 256 TMEM columns and issues the MMAs:
 //               S_{j+1} = Q K_{j+1}^T as soon as softmax has read S_j, then
 //               O += P_j V_j once P_j is in shared memory
-//               (both single-thread roles wait with a suspend-time hint)
+//               (both roles run their loop with the whole warp and issue from
+//               one elected lane; their waits carry a suspend-time hint)
 //   warps 2-3   idle
 //   warps 4-7   softmax: one query row per thread (TMEM lane), reads S with
 //               tcgen05.ld, writes P_j (swizzled, double-buffered) to shared
