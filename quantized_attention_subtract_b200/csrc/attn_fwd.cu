@@ -169,7 +169,7 @@ __device__ __forceinline__ float tile_max(uint32_t (&s)[128], float c0, float c1
 // op rounds like its scalar counterpart.
 template <int D, bool kSmoothQ>
 __device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], float c0, float c1, float nmb,
-                                          uint8_t *prow_base, int row, bool rescale, float alpha,
+                                          uint32_t prow_s, uint32_t rx, bool rescale, float alpha,
                                           uint32_t tO) {
   constexpr float kBias = 12582912.0f;
   constexpr int kChunks = D / 32;
@@ -210,10 +210,8 @@ __device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], float c0, fl
       pk[q] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
     }
     // keys 32 sec .. 32 sec + 31 are the 16-byte units 2 sec and 2 sec + 1 of the row
-    *reinterpret_cast<uint4 *>(prow_base + swz_offset(row, 32 * sec, 128)) =
-        make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<uint4 *>(prow_base + swz_offset(row, 32 * sec + 16, 128)) =
-        make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    sts128(prow_s + ((32u * sec) ^ rx), pk[0], pk[1], pk[2], pk[3]);
+    sts128(prow_s + ((32u * sec + 16u) ^ rx), pk[4], pk[5], pk[6], pk[7]);
     if (ch >= 0 && ch < kChunks && rescale) {
       tmem_ld32_wait(o);
 #pragma unroll
@@ -605,6 +603,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t lane_off = uint32_t(32 * wq) << 16;
     const uint32_t tS = tmem + lane_off, tO = tmem + lane_off + 128;
     const float qs = kFuseQ ? qs_fused : ws.q_scale[(long long)bh * nq + qt];
+    const uint32_t prow_rx = uint32_t(row & 7) << 4;   // swizzle of this row's 16-byte units
     const float *ksc = ws.k_scale + (long long)bhk * (ws.Nkv_pad / kKBlk);
     const float *dsk = kSmoothQ ? ws.dsk + ((long long)bh * nq + qt) * ws.Nkv_pad : nullptr;
     float m_run = -INFINITY, l = 0.f;
@@ -660,9 +659,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         ok = false;
         break;
       }
-      uint8_t *pbuf = smem + C::kOffP + (j & 1) * C::kPBytes;
+      // this row of P_j's buffer (128 bytes; 16-byte units XOR-swizzled by row % 8)
+      const uint32_t prow_s = sP + uint32_t(j & 1) * C::kPBytes + uint32_t(row) * 128u;
       const float a_row = need ? alpha : 1.f;
-      const float lsum = tile_exp<D, kSmoothQ>(s, c0, c1, nmb, pbuf, row, rescale, a_row, tO);
+      const float lsum = tile_exp<D, kSmoothQ>(s, c0, c1, nmb, prow_s, prow_rx, rescale, a_row, tO);
       l = __fmaf_rn(l, alpha, lsum);
       // P stores visible to the tensor core (async proxy), TMEM writes ordered,
       // then P_j is handed to the MMA warp
@@ -686,19 +686,28 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_ld32(tO + 32 * c, r);
         uint32_t packed[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float o0 = __uint_as_float(r[e]) * (__ldg(vs + 32 * c + e) * inv_l);
-          float o1 = __uint_as_float(r[e + 1]) * (__ldg(vs + 32 * c + e + 1) * inv_l);
+        for (int e = 0; e < 32; e += 4) {
+          // channel scales (and means) four at a time: the per-head arrays are
+          // 256-byte aligned and 32 c + e is a multiple of 4
+          const float4 s4 = __ldg(reinterpret_cast<const float4 *>(vs + 32 * c + e));
+          float o[4] = {__uint_as_float(r[e]) * (s4.x * inv_l), __uint_as_float(r[e + 1]) * (s4.y * inv_l),
+                        __uint_as_float(r[e + 2]) * (s4.z * inv_l), __uint_as_float(r[e + 3]) * (s4.w * inv_l)};
           if (pb.smooth_v) {
-            o0 += __ldg(mv + 32 * c + e);
-            o1 += __ldg(mv + 32 * c + e + 1);
+            const float4 m4 = __ldg(reinterpret_cast<const float4 *>(mv + 32 * c + e));
+            o[0] += m4.x;
+            o[1] += m4.y;
+            o[2] += m4.z;
+            o[3] += m4.w;
           }
-          if (pb.bf16) {
-            const __nv_bfloat162 v2 = __floats2bfloat162_rn(o0, o1);
-            packed[e / 2] = *reinterpret_cast<const uint32_t *>(&v2);
-          } else {
-            const __half2 v2 = __floats2half2_rn(o0, o1);
-            packed[e / 2] = *reinterpret_cast<const uint32_t *>(&v2);
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            if (pb.bf16) {
+              const __nv_bfloat162 v2 = __floats2bfloat162_rn(o[2 * h2], o[2 * h2 + 1]);
+              packed[e / 2 + h2] = *reinterpret_cast<const uint32_t *>(&v2);
+            } else {
+              const __half2 v2 = __floats2half2_rn(o[2 * h2], o[2 * h2 + 1]);
+              packed[e / 2 + h2] = *reinterpret_cast<const uint32_t *>(&v2);
+            }
           }
         }
         if (i < Nq_b) {

@@ -363,6 +363,12 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 16-byte store to a shared-memory address.
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 // One lane of the (converged) warp gets true: elect.sync over all 32 lanes.
 __device__ __forceinline__ bool elect_one() {
   uint32_t leader;
