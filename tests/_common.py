@@ -32,7 +32,7 @@ def to_device(bits: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
     return t.view(torch.float16 if dtype == "fp16" else torch.bfloat16)
 
 
-class GpuRun:
+class DeviceRun:
     """Inputs on the device, the output, the workspace and its views."""
 
     def __init__(self, w: Workload, q, k, v, run_attention: bool = True, fuse_q: bool = False):
@@ -58,11 +58,11 @@ def run_both(w: Workload, seed=None, fuse_q: bool = False):
     q, k, v = generate(w, seed)
     pr = oracle_problem(w)
     pre = oracle.prepass(pr, q, k, v)
-    g = GpuRun(w, q, k, v, fuse_q=fuse_q)
+    g = DeviceRun(w, q, k, v, fuse_q=fuse_q)
     return q, k, v, pr, pre, g
 
 
-def assert_prepass_bit_exact(w: Workload, pre: dict, g: GpuRun):
+def assert_prepass_bit_exact(w: Workload, pre: dict, g: DeviceRun):
     V = {k: (v.cpu().numpy() if isinstance(v, torch.Tensor) else v) for k, v in g.views.items()}
     D, Nq, Nkv = w.D, w.Nq, w.Nkv
     q8 = V["q8"]
@@ -114,7 +114,7 @@ def half_ulp(x: np.ndarray, dtype: str) -> np.ndarray:
     return h
 
 
-def compare_output(pr: oracle.Problem, pre: dict, q, k, v, g: GpuRun, tiles, exact: bool = True):
+def compare_output(pr: oracle.Problem, pre: dict, q, k, v, g: DeviceRun, tiles, exact: bool = True):
     """GPU output vs the mirror (and vs exact fp64 attention) on `tiles`.
 
     max_abs_excess is max(|gpu - mirror| - unc - half_ulp): the part of the

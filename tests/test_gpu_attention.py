@@ -12,7 +12,7 @@ import oracle
 from quantized_attention_subtract_b200 import binding, sageattn
 from quantized_attention_subtract_b200.workloads import generate, random_problem
 
-from _common import (EXACT_COS, EXACT_REL_L1, MIRROR_COS, MIRROR_MAX_ABS, GpuRun,
+from _common import (EXACT_COS, EXACT_REL_L1, MIRROR_COS, MIRROR_MAX_ABS, DeviceRun,
                      assert_prepass_bit_exact, compare_output, oracle_problem, run_both, to_device)
 
 pytestmark = pytest.mark.gpu
@@ -65,8 +65,8 @@ def test_fused_q_matches_separate_prepass(case):
     flags = {k: v for k, v in case.items() if k == "is_causal"}
     w = random_problem(*case["args"], layout=case["layout"], dtype=case["dtype"], seed=21, **flags)
     q, k, v = generate(w)
-    fused = GpuRun(w, q, k, v, fuse_q=True)
-    sep = GpuRun(w, q, k, v, run_attention=False)
+    fused = DeviceRun(w, q, k, v, fuse_q=True)
+    sep = DeviceRun(w, q, k, v, run_attention=False)
     binding.attn_quantized(sep.p, sep.q.device)
     torch.cuda.synchronize()
     assert binding.device_status(sep.p) == 0
@@ -78,7 +78,7 @@ def test_fused_q_matches_separate_prepass(case):
 def test_public_api_matches_params_path_and_host_tensors():
     w = random_problem(1, 4, 2, 300, 300, 128, dtype="bf16", seed=2)
     q, k, v = generate(w)
-    g = GpuRun(w, q, k, v)
+    g = DeviceRun(w, q, k, v)
     a = sageattn(g.q, g.k, g.v, tensor_layout="HND", is_causal=False)
     torch.cuda.synchronize()
     assert torch.equal(a, g.out)
@@ -92,7 +92,7 @@ def test_host_tensors_nhd():
     the device path's output bit for bit."""
     w = random_problem(2, 4, 2, 300, 260, 64, layout="NHD", dtype="fp16", seed=6)
     q, k, v = generate(w)
-    g = GpuRun(w, q, k, v)
+    g = DeviceRun(w, q, k, v)
     h = sageattn(g.q.cpu().pin_memory(), g.k.cpu().pin_memory(), g.v.cpu().pin_memory(),
                  tensor_layout="NHD")
     torch.cuda.synchronize()
@@ -103,7 +103,7 @@ def test_strided_inputs():
     """q, k, v as views with padded token strides (still 16-byte aligned rows)."""
     w = random_problem(1, 2, 2, 256, 256, 64, dtype="fp16", seed=5)
     q, k, v = generate(w)
-    dense = GpuRun(w, q, k, v)
+    dense = DeviceRun(w, q, k, v)
     big = torch.zeros(1, 2, 256, 128, dtype=torch.float16, device="cuda")
     views = []
     for t in (dense.q, dense.k, dense.v):
@@ -136,7 +136,7 @@ def test_constant_v_rows_give_the_constant():
     import torch as _t
     vb = _t.from_numpy(np.broadcast_to(const, (1, 2, 700, 128)).copy()).to(_t.bfloat16)
     v = vb.view(_t.int16).numpy().view(np.uint16)
-    g = GpuRun(w, q, k, v)
+    g = DeviceRun(w, q, k, v)
     c = vb[0, 0, 0].double().numpy()
     o = g.out_f64()
     assert np.all(np.abs(o - c) <= 2.0 ** -4 * np.abs(c) + 2 ** -8)

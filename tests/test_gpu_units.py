@@ -16,7 +16,7 @@ import oracle
 from quantized_attention_subtract_b200 import binding
 from quantized_attention_subtract_b200.workloads import generate, random_problem
 
-from _common import GpuRun, oracle_problem
+from _common import DeviceRun, oracle_problem
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +54,7 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     torch.cuda.synchronize()
     assert int(st[0]) == 5  # SAGE_ERR_DEVICE_TIMEOUT
     w = random_problem(1, 2, 2, 128, 128, 64, seed=1)
-    g = GpuRun(w, *generate(w))
+    g = DeviceRun(w, *generate(w))
     assert torch.isfinite(g.out.float()).all()
 
 
@@ -64,7 +64,7 @@ def test_s_tiles_bit_exact(D, Nq, Nkv, layout):
     w = random_problem(2, 4, 2, Nq, Nkv, D, layout=layout, dtype="bf16", seed=D)
     q, k, v = generate(w)
     pre = oracle.prepass(oracle_problem(w), q, k, v)
-    g = GpuRun(w, q, k, v, run_attention=False)
+    g = DeviceRun(w, q, k, v, run_attention=False)
     nqt, nkt = (Nq + 127) // 128, (Nkv + 127) // 128
     for b, h, qt, kt in [(0, 0, 0, 0), (1, 3, nqt - 1, nkt - 1), (0, 2, nqt - 1, 0), (1, 1, 0, nkt - 1)]:
         s = binding.debug_dump_s(g.p, b, h, qt, kt, "cuda").cpu().numpy().astype(np.int64)
@@ -82,7 +82,7 @@ def test_pv_tile_fp32_accumulation(D):
     w = random_problem(1, 1, 1, 128, 256, D, dtype="fp16", seed=3)
     q, k, v = generate(w)
     pre = oracle.prepass(oracle_problem(w), q, k, v)
-    g = GpuRun(w, q, k, v, run_attention=False)
+    g = DeviceRun(w, q, k, v, run_attention=False)
     rng = np.random.default_rng(D)
     table = oracle.e4m3_decode_table()
     # random non-negative finite codes, as P is
