@@ -389,13 +389,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = align1024(smem_raw);
-  const uint32_t s_base = smem_u32(smem);
+  // the shared base, the warp index and (below) the TMEM base go through a
+  // shuffle from lane 0, so the compiler knows them warp-uniform and keeps
+  // the barrier and TMEM addresses built from them in uniform registers
+  const uint32_t s_base = __shfl_sync(0xffffffffu, smem_u32(smem), 0);
   const uint32_t sQ = s_base + C::kOffQ, sRing = s_base + C::kOffRing, sP = s_base + C::kOffP;
   const uint32_t bars = s_base + C::kOffBar;
   auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffBar + 8 * kNumBars);
 
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int warp = __shfl_sync(0xffffffffu, int(threadIdx.x / 32), 0), lane = threadIdx.x % 32;
   int *status = ws.status;
 
   // ---- work item: (b, h, query tile); causal runs the longest tiles first
@@ -438,7 +441,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   const bool skip_all = *(volatile int *)status != 0;  // an earlier CTA already failed
 
   // ---- producer (thread 0) state: with fused Q the first ring loads are
