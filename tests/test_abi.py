@@ -215,3 +215,25 @@ def test_host_chunks_cover_every_head_once_in_contiguous_slices(layout, B, Hkv, 
         else:
             view = q[b:b + 1, :, h0 * group:h1 * group]
         assert view.is_contiguous(), (b, h0, h1)
+
+
+@pytest.mark.parametrize("kw,code", [
+    # 32-bit TMA row coordinates and kernel indices: B * H * (N rounded up to 128) < 2^31
+    (dict(Hq=2, Hkv=2, Nq=(1 << 30) - 128, Nkv=256), 0),
+    (dict(Hq=2, Hkv=2, Nq=(1 << 30) - 127, Nkv=256), 2),
+    (dict(Hq=2, Hkv=2, Nq=256, Nkv=(1 << 30) - 128), 0),
+    (dict(Hq=2, Hkv=2, Nq=256, Nkv=1 << 30), 2),
+    (dict(B=(1 << 17) - 1, Hq=128, Hkv=128, Nq=128, Nkv=128), 0),
+    (dict(B=1 << 17, Hq=128, Hkv=128, Nq=128, Nkv=128), 2),
+])
+def test_size_limits(kw, code):
+    """The largest problems the 32-bit indices allow are accepted and one
+    128-row tile more is rejected as unsupported, before any device work."""
+    assert _ws_size(_params(**kw))[0] == code
+
+
+@pytest.mark.parametrize("scale", [float("nan"), float("inf"), float("-inf")])
+def test_non_finite_sm_scale_rejected(scale):
+    p = _params()
+    p.sm_scale = scale
+    assert _ws_size(p)[0] == 1
