@@ -16,7 +16,9 @@
  *      tokens) with fp32 scales; V to FP8 e4m3 with per-channel scales;
  *   3. a flash-style kernel: INT8 Q K^T with exact int32 accumulation,
  *      dequantisation, online softmax (running max and sum, exp2), P
- *      quantised to FP8 e4m3 as 448 * exp2(s - m), FP8 P V with fp32
+ *      quantised to FP8 e4m3 as 224 * exp2(s - m), where m is a per-row
+ *      reference max raised to a tile's max only when that exceeds m by more
+ *      than 1 (so every value stays within e4m3's 448), FP8 P V with fp32
  *      accumulation;
  *   4. epilogue: divide by the row sum, rescale by the V channel scale (and
  *      add the V mean back), round to the input's 16-bit type.
@@ -30,7 +32,13 @@
  *   - Every internal wait of the kernels is bounded (about one second).  A
  *     wait that runs out records SAGE_ERR_DEVICE_TIMEOUT in the workspace's
  *     status word and the kernel returns early; read it with
- *     sage_get_device_status() after the stream has finished.
+ *     sage_get_device_status() after the stream has finished.  A pre-pass
+ *     kernel whose shared memory is not 128-byte aligned (not expected)
+ *     records SAGE_ERR_ALIGNMENT there and does nothing.
+ *   - Sizes: B * Hq * Nq and B * Hkv * Nkv, with Nq and Nkv rounded up to
+ *     128, and B * Hkv * D must stay below 2^31 (32-bit tensor-map
+ *     coordinates and kernel indices); larger problems are rejected with
+ *     SAGE_ERR_UNSUPPORTED.
  */
 #ifndef SAGE_B200_H
 #define SAGE_B200_H
