@@ -25,9 +25,10 @@ _SRC = os.path.join(_HERE, "sage_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _SO = os.path.join(_BUILD, "liboracle.so")
 
-QBLK = 128
-KBLK = 64
-KVT = 128
+QTILE = 128   # query rows per output tile
+QMBLK = 128   # query smoothing-mean block (tokens)
+KBLK = 32     # key quantisation block (tokens)
+KVT = 128     # keys per online-softmax tile
 
 _lock = threading.Lock()
 _lib = None
@@ -59,8 +60,8 @@ def _load():
             lib = ctypes.CDLL(build())
             P = ctypes.POINTER(_Params)
             vp = ctypes.c_void_p
-            lib.oracle_prepass.argtypes = [P] + [vp] * 13
-            lib.oracle_attention_tiles.argtypes = [P] + [vp] * 9 + [ctypes.c_int, vp, vp, vp]
+            lib.oracle_prepass.argtypes = [P] + [vp] * 15
+            lib.oracle_attention_tiles.argtypes = [P] + [vp] * 11 + [ctypes.c_int, ctypes.c_int, vp, vp, vp]
             lib.oracle_exact_attention_tiles.argtypes = [P, vp, vp, vp, ctypes.c_int, vp, vp]
             lib.oracle_round_output.argtypes = [P, vp, vp, ctypes.c_int64]
             lib.oracle_e4m3_encode_array.argtypes = [vp, vp, ctypes.c_int64]
@@ -112,7 +113,13 @@ class Problem:
 
     @property
     def nqb(self) -> int:
-        return (self.Nq + QBLK - 1) // QBLK
+        """Query tiles of 128 rows (the output tiling)."""
+        return (self.Nq + QTILE - 1) // QTILE
+
+    @property
+    def nmb(self) -> int:
+        """Query smoothing-mean blocks of 128 tokens."""
+        return (self.Nq + QMBLK - 1) // QMBLK
 
     @property
     def nkb(self) -> int:
@@ -129,8 +136,13 @@ def _ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
-def prepass(pr: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
-    """Smoothing + quantisation of Q, K, V (all heads). Inputs: uint16 bit patterns."""
+def prepass(pr: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray,
+            keep_fp32: bool = False) -> dict:
+    """Smoothing + quantisation of Q, K, V (all heads). Inputs: uint16 bit patterns.
+
+    q_scale holds one scale per query token, k_scale one per 32 keys.  With
+    keep_fp32 the smoothed fp32 inputs Q' (qp) and V' (vp) are returned too
+    (the unquantised operands of the error decomposition)."""
     lib = _load()
     q, k, v = _bits(q), _bits(k), _bits(v)
     B, Hq, Hkv, Nq, Nkv, D = pr.B, pr.Hq, pr.Hkv, pr.Nq, pr.Nkv, pr.D
@@ -139,17 +151,21 @@ def prepass(pr: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarray) -> dict:
         kp=np.zeros((B, Hkv, Nkv, D), np.float32),
         k8=np.zeros((B, Hkv, Nkv, D), np.int8),
         k_scale=np.zeros((B, Hkv, pr.nkb), np.float32),
-        mq=np.zeros((B, Hq, pr.nqb, D), np.float32),
+        mq=np.zeros((B, Hq, pr.nmb, D), np.float32),
         q8=np.zeros((B, Hq, Nq, D), np.int8),
-        q_scale=np.zeros((B, Hq, pr.nqb), np.float32),
+        q_scale=np.zeros((B, Hq, Nq), np.float32),
         mean_v=np.zeros((B, Hkv, D), np.float32),
         v8=np.zeros((B, Hkv, Nkv, D), np.uint8),
         v_scale=np.zeros((B, Hkv, D), np.float32),
     )
+    if keep_fp32:
+        out["qp"] = np.zeros((B, Hq, Nq, D), np.float32)
+        out["vp"] = np.zeros((B, Hkv, Nkv, D), np.float32)
     c = pr._c()
     lib.oracle_prepass(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v),
                        *[_ptr(out[n]) for n in ("mean_k", "kp", "k8", "k_scale", "mq", "q8",
-                                                "q_scale", "mean_v", "v8", "v_scale")])
+                                                "q_scale", "mean_v", "v8", "v_scale")],
+                       _ptr(out["qp"]) if keep_fp32 else None, _ptr(out["vp"]) if keep_fp32 else None)
     return out
 
 
@@ -158,21 +174,32 @@ def all_tiles(pr: Problem) -> np.ndarray:
                     np.int32).reshape(-1, 3)
 
 
-def attention_tiles(pr: Problem, pre: dict, tiles, with_uncertainty: bool = False):
-    """Mirror of the tiled quantised attention for (b, h, q_tile) triples.
+KEEP_P, KEEP_V, KEEP_QK = 1, 2, 4
+
+
+def attention_tiles(pr: Problem, pre: dict, tiles, with_uncertainty: bool = False,
+                    exact_mask: int = 0):
+    """The tiled quantised attention (the plain online softmax) for
+    (b, h, q_tile) triples.
 
     Returns fp64 [n_tiles, 128, D] (rows past Nq are zero); with
-    `with_uncertainty`, also the per-element bound of how far an
-    implementation may differ because an FP8 code of P sits within the exp2
-    error band of an e4m3 rounding midpoint (see sage_oracle.c).
+    `with_uncertainty`, also the per-element bound of how far an fp32
+    implementation may differ because an FP8 code of P sits within its
+    rounding band of an e4m3 midpoint (see sage_oracle.c).  exact_mask
+    (KEEP_P | KEEP_V | KEEP_QK) leaves those steps unquantised, for the error
+    decomposition; KEEP_V and KEEP_QK need a pre-pass run with keep_fp32.
     """
     lib = _load()
     tiles = np.ascontiguousarray(np.asarray(tiles, np.int32).reshape(-1, 3))
-    out = np.zeros((len(tiles), QBLK, pr.D), np.float64)
+    out = np.zeros((len(tiles), QTILE, pr.D), np.float64)
     unc = np.zeros_like(out) if with_uncertainty else None
+    if exact_mask & (KEEP_V | KEEP_QK):
+        assert "qp" in pre and "vp" in pre, "run prepass(..., keep_fp32=True)"
     c = pr._c()
     names = ("q8", "q_scale", "k8", "k_scale", "v8", "v_scale", "mean_v", "mq", "kp")
     lib.oracle_attention_tiles(ctypes.byref(c), *[_ptr(pre[n]) for n in names],
+                               _ptr(pre["qp"]) if "qp" in pre else None,
+                               _ptr(pre["vp"]) if "vp" in pre else None, int(exact_mask),
                                len(tiles), _ptr(tiles), _ptr(out),
                                _ptr(unc) if unc is not None else None)
     return (out, unc) if with_uncertainty else out
@@ -183,7 +210,7 @@ def exact_attention_tiles(pr: Problem, q: np.ndarray, k: np.ndarray, v: np.ndarr
     lib = _load()
     q, k, v = _bits(q), _bits(k), _bits(v)
     tiles = np.ascontiguousarray(np.asarray(tiles, np.int32).reshape(-1, 3))
-    out = np.zeros((len(tiles), QBLK, pr.D), np.float64)
+    out = np.zeros((len(tiles), QTILE, pr.D), np.float64)
     c = pr._c()
     lib.oracle_exact_attention_tiles(ctypes.byref(c), _ptr(q), _ptr(k), _ptr(v), len(tiles),
                                      _ptr(tiles), _ptr(out))
@@ -232,9 +259,9 @@ def tile_rows(pr: Problem, tiles, x: np.ndarray):
     """Gather rows of an [.., D] output in (b, h, q_tile) tiling: returns [n, 128, D]
     (rows past Nq zero).  `x` is a full output in the problem's layout."""
     tiles = np.asarray(tiles, np.int32).reshape(-1, 3)
-    out = np.zeros((len(tiles), QBLK, pr.D), x.dtype)
+    out = np.zeros((len(tiles), QTILE, pr.D), x.dtype)
     for n, (b, h, t) in enumerate(tiles):
-        i0, i1 = t * QBLK, min(t * QBLK + QBLK, pr.Nq)
+        i0, i1 = t * QTILE, min(t * QTILE + QTILE, pr.Nq)
         if pr.layout == "HND":
             out[n, : i1 - i0] = x[b, h, i0:i1]
         else:
@@ -243,7 +270,8 @@ def tile_rows(pr: Problem, tiles, x: np.ndarray):
 
 
 def delta_s(pr: Problem, pre: dict, b: int, h: int, qt: int) -> np.ndarray:
-    """Q-smoothing correction row dS[j] = mq(b,h,qt) . K'(b,kv(h),j) in fp64."""
+    """Q-smoothing correction row dS[j] = mq(b,h,qt) . K'(b,kv(h),j) in fp64
+    (qt indexes the 128-token smoothing-mean blocks)."""
     lib = _load()
     lib.oracle_delta_s.argtypes = [ctypes.POINTER(_Params), ctypes.c_void_p, ctypes.c_void_p,
                                    ctypes.c_void_p]
@@ -299,7 +327,7 @@ def varlen_attention(Hq: int, Hkv: int, D: int, cu_q, cu_kv, q: np.ndarray, k: n
         if exact:
             parts["exact"] = exact_attention_tiles(pr, qs, ks, vs, tiles)
         for n, (_, h, t) in enumerate(tiles):
-            i0, i1 = t * QBLK, min(t * QBLK + QBLK, pr.Nq)
+            i0, i1 = t * QTILE, min(t * QTILE + QTILE, pr.Nq)
             for name, arr in parts.items():
                 if arr is not None:
                     res[name][q0 + i0:q0 + i1, h] = arr[n, :i1 - i0]

@@ -14,41 +14,44 @@
  *     "What it is": per-block quantization of queries and keys plus
  *     smoothing; head dims 64/96/128, Nq != Nkv, group-query attention.
  *   - closerAI ComfyUI blog, part 2 ("keeping precision"): INT8 for QK^T,
- *     FP8 for PV, smoothing to reduce quantisation error.
- *   - "SageAttention2: Technical report" (ai-digest.ru), section 2
- *     ("smoothing Q and V"): the channel mean of Q and V is subtracted
- *     before quantisation.
+ *     FP8 for PV, smoothing to reduce quantisation error, quantisation at
+ *     several granularities; part 4: SageAttention2's per-thread
+ *     quantisation, finer than per block.
+ *   - "SageAttention2: Technical report" (ai-digest.ru), section 1: Q and K
+ *     quantised at warp / thread granularity; section 2 ("smoothing Q and
+ *     V"): the channel mean of Q and V is subtracted before quantisation.
  *   - The flash-style tiled pass (online softmax with running max and sum,
  *     exp2, P quantised to FP8, FP32 accumulation) is the FlashAttention
  *     comparison all pages make (e.g. the pwwt.cn guide, section 3.2).
  *
  * The pages fix no block size, rounding rule or scale convention.  The
- * readings taken here (each also a constant of the CUDA path, so both sides
- * agree by construction) are:
- *   - Q blocks of 128 tokens, K blocks of 64 tokens, KV tiles of 128 keys.
+ * readings taken here are:
+ *   - Q is quantised with one INT8 scale per query token (per-thread
+ *     granularity where one thread owns one query row); K with one scale per
+ *     block of 32 keys; the online softmax walks KV tiles of 128 keys.
  *   - INT8 codes are symmetric in [-127, 127]: scale = amax/127,
  *     code = rint(x * (127/amax)) with round-half-even, computed in IEEE
  *     fp32 without FMA contraction.  A block with amax < 2^-64 gets scale 0
  *     and all-zero codes.
  *   - Means are exact fixed-point means: sum of rint(x * 2^24) in int64,
  *     divided in fp64 by n * 2^24 and rounded to fp32.  This makes the mean
- *     independent of summation order.
+ *     independent of summation order.  Q's smoothing mean is taken per block
+ *     of 128 tokens.
  *   - V is FP8 e4m3 per channel over all tokens: scale = amax/448, code =
  *     e4m3_rn_satfinite(x * (448/amax)).
- *   - Online softmax keeps, per row, a reference max m that is raised to a
- *     tile's max only when that exceeds m by more than one binade (fp32
- *     test t_max > m + 1); O and l are rescaled by 2^(m_old - m_new) only
- *     then.  Every logit of a tile that did not raise m is <= m + 1, so P is
- *     quantised as e4m3(224 * 2^(s - m)), which never exceeds 448 (e4m3's
- *     largest finite value).  The row sum l accumulates the unquantised
- *     values; O accumulates the quantised ones.
+ *   - Online softmax, the plain definition: per KV tile the row's running
+ *     max m becomes max(m, tile max); when it grows, O and l are multiplied
+ *     by 2^(m_old - m_new); every visible key contributes
+ *     p = 448 * 2^(s - m) to l unquantised and, quantised to e4m3, to
+ *     O += e4m3(p) * v.  p <= 448, e4m3's largest finite value.
  *   - Causal masking is top-left aligned (key j is visible to query i when
  *     j <= i), as in scaled_dot_product_attention.
  *   - Query head h reads kv head h / (Hq / Hkv).
  *
- * Floating point: the steps whose result is an integer code (Q/K/V
- * quantisation, the FP8 code of P) are taken in fp32, the precision of the
- * CUDA path; everything else is fp64.  Build with -ffp-contract=off and no
+ * Floating point: the quantisation steps whose result is an integer code
+ * (INT8 of Q and K, FP8 of V) are taken in fp32, the precision of the CUDA
+ * path.  The logits s = S * q_scale * k_scale * sm_scale * log2(e) and
+ * everything after them are fp64.  Build with -ffp-contract=off and no
  * -ffast-math so that every fp32 operation here is one IEEE-rounded op.
  */
 #include <math.h>
@@ -60,9 +63,10 @@
 #include <omp.h>
 #endif
 
-#define QBLK 128   /* query quantisation block (tokens) */
-#define KBLK 64    /* key quantisation block (tokens)   */
-#define KVT 128    /* keys per online-softmax tile      */
+#define QMBLK 128  /* query smoothing-mean block (tokens)  */
+#define KBLK 32    /* key quantisation block (tokens)     */
+#define KVT 128    /* keys per online-softmax tile        */
+#define QTILE 128  /* query rows per output tile          */
 
 typedef struct {
     int B, Hq, Hkv, Nq, Nkv, D;
@@ -217,20 +221,22 @@ static float quantise_int8_block(const float *x, int64_t n, int8_t *codes) {
  * Outputs (natural layouts, independent of the input layout):
  *   mean_k  f32 [B][Hkv][D]          (zeros when smooth_k == 0)
  *   kp      f32 [B][Hkv][Nkv][D]     K' = K - mean_k (fp32)
- *   k8      i8  [B][Hkv][Nkv][D];  k_scale f32 [B][Hkv][ceil(Nkv/64)]
- *   mq      f32 [B][Hq][nqb][D]      (zeros when smooth_q == 0)
- *   q8      i8  [B][Hq][Nq][D];    q_scale f32 [B][Hq][nqb]
+ *   k8      i8  [B][Hkv][Nkv][D];  k_scale f32 [B][Hkv][ceil(Nkv/32)]
+ *   mq      f32 [B][Hq][ceil(Nq/128)][D]   (zeros when smooth_q == 0)
+ *   q8      i8  [B][Hq][Nq][D];    q_scale f32 [B][Hq][Nq]  (one per token)
  *   mean_v  f32 [B][Hkv][D]          (zeros when smooth_v == 0)
  *   v8      u8  [B][Hkv][Nkv][D];  v_scale f32 [B][Hkv][D]
+ *   qp      f32 [B][Hq][Nq][D]       Q' = Q - mq (fp32); may be NULL
+ *   vp      f32 [B][Hkv][Nkv][D]     V' = V - mean_v (fp32); may be NULL
  * ------------------------------------------------------------------- */
 void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k,
                     const uint16_t *v, float *mean_k, float *kp, int8_t *k8,
                     float *k_scale, float *mq, int8_t *q8, float *q_scale,
-                    float *mean_v, uint8_t *v8, float *v_scale) {
+                    float *mean_v, uint8_t *v8, float *v_scale, float *qp, float *vp_out) {
     const int D = p->D, Nq = p->Nq, Nkv = p->Nkv;
-    const int nqb = (Nq + QBLK - 1) / QBLK, nkb = (Nkv + KBLK - 1) / KBLK;
+    const int nmb = (Nq + QMBLK - 1) / QMBLK, nkb = (Nkv + KBLK - 1) / KBLK;
 
-    /* K: mean over all tokens, K' = K - mean, per-64-token INT8 blocks. */
+    /* K: mean over all tokens, K' = K - mean, per-32-token INT8 blocks. */
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < p->B; b++)
         for (int h = 0; h < p->Hkv; h++) {
@@ -251,22 +257,26 @@ void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k
             free(col);
         }
 
-    /* Q: optional per-block mean, Q' = Q - mq, per-128-token INT8 blocks. */
+    /* Q: optional per-128-token block mean, Q' = Q - mq, one INT8 scale per
+     * token (the token's D channels form its quantisation block). */
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < p->B; b++)
         for (int h = 0; h < p->Hq; h++) {
-            float *blk = (float *)malloc(sizeof(float) * QBLK * (size_t)D);
-            double *col = (double *)malloc(sizeof(double) * QBLK);
-            for (int qb = 0; qb < nqb; qb++) {
-                int i0 = qb * QBLK, n = (Nq - i0 < QBLK) ? Nq - i0 : QBLK;
-                float *mqb = mq + (((int64_t)b * p->Hq + h) * nqb + qb) * D;
+            float *blk = (float *)malloc(sizeof(float) * QMBLK * (size_t)D);
+            double *col = (double *)malloc(sizeof(double) * QMBLK);
+            for (int mb = 0; mb < nmb; mb++) {
+                int i0 = mb * QMBLK, n = (Nq - i0 < QMBLK) ? Nq - i0 : QMBLK;
+                float *mqb = mq + (((int64_t)b * p->Hq + h) * nmb + mb) * D;
                 for (int c = 0; c < D; c++) {
                     for (int r = 0; r < n; r++) col[r] = in_to_double(p, q[idx(p, p->Hq, Nq, b, h, i0 + r, c)]);
                     mqb[c] = p->smooth_q ? fixed_point_mean(col, n) : 0.0f;
                     for (int r = 0; r < n; r++) blk[(int64_t)r * D + c] = (float)col[r] - mqb[c];
                 }
-                q_scale[((int64_t)b * p->Hq + h) * nqb + qb] = quantise_int8_block(
-                    blk, (int64_t)n * D, q8 + (((int64_t)b * p->Hq + h) * Nq + i0) * D);
+                for (int r = 0; r < n; r++) {
+                    const int64_t row = ((int64_t)b * p->Hq + h) * Nq + i0 + r;
+                    q_scale[row] = quantise_int8_block(blk + (int64_t)r * D, D, q8 + row * D);
+                    if (qp) memcpy(qp + row * D, blk + (int64_t)r * D, sizeof(float) * (size_t)D);
+                }
             }
             free(blk);
             free(col);
@@ -286,6 +296,7 @@ void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k
                 for (int j = 0; j < Nkv; j++) {
                     vp[j] = (float)col[j] - mv;
                     if (fabsf(vp[j]) > amax) amax = fabsf(vp[j]);
+                    if (vp_out) vp_out[(((int64_t)b * p->Hkv + h) * Nkv + j) * D + c] = vp[j];
                 }
                 uint8_t *v8h = v8 + ((int64_t)b * p->Hkv + h) * Nkv * D;
                 if (!(amax >= 0x1p-64f)) {
@@ -320,144 +331,166 @@ void oracle_delta_s(const oracle_params *p, const float *mq_blk, const float *kp
  * The tiled quantised attention, step by step, for selected query tiles.
  *
  * tiles: n_tiles triples (b, h, qt); out: [n_tiles][128][D] fp64 outputs
- * (rows >= Nq are left untouched).  S is formed in int64 from the codes;
- * per 128-key tile the row logits are s = S * c_half with
- * c_half = (q_scale * k_scale[half]) * K2, K2 = fl32(sm_scale * fl32(log2 e)),
- * all in fp32; the reference max m (raised lazily, see above) and the
- * shifted max mb = m - fl32(log2 224) are fp32; the exponent is the fused
- * fp32 t = S * c - mb; p = 2^t in fp64, rounded to fp32 (flushing results
- * below 2^-126 to zero); P8 = e4m3(p).  l (fp64) accumulates p, O (fp64)
- * accumulates decode(P8) * decode(v8), and both are multiplied by
- * 2^(m_old - m_new) when m is raised.
- * Output o = O * v_scale / l (+ mean_v).
+ * (rows >= Nq are left untouched).  Per row i and 128-key tile:
+ *   S_j  = q8_i . k8_j in int64 (exact);
+ *   s_j  = S_j * q_scale_i * k_scale_blk(j) * sm_scale * log2(e)
+ *          (+ dS_j * sm_scale * log2(e) with smoothed Q), in fp64 from the
+ *          fp32 scales;
+ *   m    = max(m, max_j s_j); when m grows, O and l *= 2^(m_old - m_new);
+ *   p_j  = 448 * 2^(s_j - m);  l += p_j;  O += e4m3(p_j) * v8_j;
+ * and finally o = O * v_scale / l (+ mean_v).
+ *
+ * exact_mask (for the error decomposition; 0 in every parity use):
+ *   bit 0: P enters O unquantised (O += p_j * v)
+ *   bit 1: V unquantised (v = V' in fp32, and no v_scale)
+ *   bit 2: Q K^T unquantised (s_j from Q' . K' in fp64; needs qp)
+ * With all three set the result is exact softmax attention of (Q, K', V)
+ * up to the fp32 rounding of the smoothed inputs.
  *
  * unc (optional, same shape as out): how far an implementation may lie from
- * `out` because the FP8 code of P is not unique.  The logit t is fixed to the
- * bit by the steps above, but the pages fix no exp2 implementation; a fast
- * hardware exp2 has a relative error of about 2^-22, so wherever 2^t lies
- * within a relative band EXP2_BAND of an e4m3 rounding midpoint, both
- * neighbouring codes are valid.  unc accumulates, per output channel, the
- * effect of taking the other code: |step| * |v8| * v_scale / l.  With
- * smoothed Q the correction dS enters t in fp32 on a GPU (fp64 here), so the
- * band widens to EXP2_BAND_SMOOTH_Q.
+ * `out` because the FP8 code of P is not unique when p is computed in fp32
+ * with a hardware exp2.  Such an implementation forms the exponent from fp32
+ * scales and logits (a few IEEE roundings, each at most 2^-24 relative:
+ * the scale product, the logit, the running max, its shift by log2(448),
+ * the subtraction; and, with smoothed Q, an fp32 dot product of D terms for
+ * dS), then a hardware exp2 of relative error at most EXP2_REL.  The first-
+ * order bound on the exponent's error, doubled, gives a relative band on p;
+ * wherever p lies within that band of an e4m3 rounding midpoint both
+ * neighbouring codes are valid, and unc accumulates, per output channel,
+ * the effect of taking the other code: |step| * |v8| * v_scale / l.
  * ------------------------------------------------------------------- */
-#define EXP2_BAND 0x1p-19
-#define EXP2_BAND_SMOOTH_Q 0x1p-12
+#define EXP2_REL 0x1p-21   /* hardware exp2 allowance (measured on the GPU by a test) */
+#define U32 0x1p-24        /* fp32 unit roundoff */
+
 void oracle_attention_tiles(const oracle_params *p, const int8_t *q8, const float *q_scale,
                             const int8_t *k8, const float *k_scale, const uint8_t *v8,
                             const float *v_scale, const float *mean_v, const float *mq,
-                            const float *kp, int n_tiles, const int *tiles, double *out,
-                            double *unc) {
+                            const float *kp, const float *qp, const float *vp, int exact_mask,
+                            int n_tiles, const int *tiles, double *out, double *unc) {
     const int D = p->D, Nq = p->Nq, Nkv = p->Nkv;
-    const int nqb = (Nq + QBLK - 1) / QBLK, nkb = (Nkv + KBLK - 1) / KBLK;
+    const int nmb = (Nq + QMBLK - 1) / QMBLK, nkb = (Nkv + KBLK - 1) / KBLK;
     const int nkt = (Nkv + KVT - 1) / KVT;
-    const float log2e = 1.44269504088896340736f;
-    const float K2 = p->sm_scale * log2e;
-    const float LP = (float)log2(224.0);   /* P scale 224 = 448 / 2 */
-    const float LAZY = 1.0f;               /* raise m only past m + 1 */
+    const double scl = (double)p->sm_scale * 1.44269504088896340736;  /* sm_scale * log2(e) */
+    const double LN2 = 0.69314718055994530942;
+    const int keep_p = exact_mask & 1, keep_v = exact_mask & 2, keep_qk = exact_mask & 4;
     double vdec[256];
     for (int c = 0; c < 256; c++) vdec[c] = oracle_e4m3_decode((uint8_t)c);
 
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int t = 0; t < n_tiles; t++)
-        for (int r = 0; r < QBLK; r++) {
+        for (int r = 0; r < QTILE; r++) {
             const int b = tiles[3 * t], h = tiles[3 * t + 1], qt = tiles[3 * t + 2];
-            const int i = qt * QBLK + r;
+            const int i = qt * QTILE + r;
             if (i >= Nq) continue;
             const int hk = h / (p->Hq / p->Hkv);
-            const float qs = q_scale[((int64_t)b * p->Hq + h) * nqb + qt];
-            const int8_t *qrow = q8 + (((int64_t)b * p->Hq + h) * Nq + i) * D;
+            const int64_t qrow_i = ((int64_t)b * p->Hq + h) * Nq + i;
+            const double qs = (double)q_scale[qrow_i];
+            const int8_t *qrow = q8 + qrow_i * D;
+            const float *qprow = qp ? qp + qrow_i * D : NULL;
             const int8_t *kh = k8 + ((int64_t)b * p->Hkv + hk) * Nkv * D;
+            const float *kph = kp + ((int64_t)b * p->Hkv + hk) * Nkv * D;
             const uint8_t *vh = v8 + ((int64_t)b * p->Hkv + hk) * Nkv * D;
+            const float *vph = vp ? vp + ((int64_t)b * p->Hkv + hk) * Nkv * D : NULL;
             const float *ksh = k_scale + ((int64_t)b * p->Hkv + hk) * nkb;
             double *O = (double *)calloc((size_t)D, sizeof(double));
             double *U = (double *)calloc((size_t)D, sizeof(double));
-            const double band = p->smooth_q ? EXP2_BAND_SMOOTH_Q : EXP2_BAND;
-            double *dS = NULL;
+            double *dS = NULL, *dmag = NULL;
+            const float *mqb = NULL;
             if (p->smooth_q) {
+                mqb = mq + (((int64_t)b * p->Hq + h) * nmb + i / QMBLK) * D;
                 dS = (double *)malloc(sizeof(double) * (size_t)Nkv);
-                oracle_delta_s(p, mq + (((int64_t)b * p->Hq + h) * nqb + qt) * D,
-                               kp + ((int64_t)b * p->Hkv + hk) * Nkv * D, dS);
+                dmag = (double *)malloc(sizeof(double) * (size_t)Nkv);
+                oracle_delta_s(p, mqb, kph, dS);
+                for (int j = 0; j < Nkv; j++) {
+                    double a = 0.0;
+                    for (int c = 0; c < D; c++) a += fabs((double)mqb[c] * (double)kph[(int64_t)j * D + c]);
+                    dmag[j] = a;
+                }
             }
-            float m_run = -INFINITY;
-            double l = 0.0;
-            int64_t S[KVT];
-            float x[KVT];
+            double m = -INFINITY, l = 0.0;
+            double s[KVT], mag[KVT];
             int valid[KVT];
             for (int kt = 0; kt < nkt; kt++) {
-                float c[2];
-                for (int hf = 0; hf < 2; hf++) {
-                    int kb = 2 * kt + hf;
-                    float ks = kb < nkb ? ksh[kb] : 0.0f;
-                    float qk = qs * ks;
-                    c[hf] = qk * K2;
-                }
-                float m_tile = -INFINITY;
+                /* logits of the tile's visible keys */
+                double tile_max = -INFINITY;
                 int any = 0;
                 for (int jj = 0; jj < KVT; jj++) {
-                    int j = kt * KVT + jj;
+                    const int j = kt * KVT + jj;
                     valid[jj] = j < Nkv && (!p->is_causal || j <= i);
                     if (!valid[jj]) continue;
                     any = 1;
-                    int64_t acc = 0;
-                    for (int cc = 0; cc < D; cc++) acc += (int64_t)qrow[cc] * (int64_t)kh[(int64_t)j * D + cc];
-                    S[jj] = acc;
-                    float sf = (float)acc;
-                    float ch = c[jj / KBLK];
-                    if (p->smooth_q) {
-                        float dsk = (float)dS[j] * K2;
-                        x[jj] = fmaf(sf, ch, dsk);
+                    double x;
+                    if (keep_qk) {
+                        double acc = 0.0;
+                        for (int c = 0; c < D; c++) acc += (double)qprow[c] * (double)kph[(int64_t)j * D + c];
+                        x = acc * scl;
                     } else {
-                        x[jj] = sf * ch;
+                        int64_t acc = 0;
+                        for (int c = 0; c < D; c++) acc += (int64_t)qrow[c] * (int64_t)kh[(int64_t)j * D + c];
+                        x = (double)acc * qs * (double)ksh[j / KBLK] * scl;
                     }
-                    if (x[jj] > m_tile) m_tile = x[jj];
+                    mag[jj] = fabs(x);
+                    if (p->smooth_q) {
+                        x += dS[j] * scl;
+                        mag[jj] += fabs(dS[j] * scl) + (double)(D + 2) * dmag[j] * scl;
+                    }
+                    s[jj] = x;
+                    if (x > tile_max) tile_max = x;
                 }
                 if (!any) continue;
-                if (m_run == -INFINITY || m_tile > m_run + LAZY) {
-                    if (m_run != -INFINITY) {
-                        const double alpha = exp2((double)m_run - (double)m_tile);
+                if (tile_max > m) {
+                    if (m != -INFINITY) {
+                        const double alpha = exp2(m - tile_max);
                         l *= alpha;
                         for (int cc = 0; cc < D; cc++) {
                             O[cc] *= alpha;
                             U[cc] *= alpha;
                         }
                     }
-                    m_run = m_tile;
+                    m = tile_max;
                 }
-                float mb = m_run - LP;
                 for (int jj = 0; jj < KVT; jj++) {
                     if (!valid[jj]) continue;
-                    int j = kt * KVT + jj;
-                    float tt;
-                    if (p->smooth_q) tt = x[jj] - mb;
-                    else tt = fmaf((float)S[jj], c[jj / KBLK], -mb);
-                    float pf = (float)exp2((double)tt);
-                    if (pf < FLT_MIN) pf = 0.0f;
-                    l += (double)pf;
-                    const uint8_t code = oracle_e4m3_encode((double)pf);
-                    double pq = vdec[code];
-                    const uint8_t *vrow = vh + (int64_t)j * D;
-                    for (int cc = 0; cc < D; cc++) O[cc] += pq * vdec[vrow[cc]];
-                    if (unc) {
-                        const double lo = vdec[oracle_e4m3_encode((double)pf * (1.0 - band))];
-                        const double hi = vdec[oracle_e4m3_encode((double)pf * (1.0 + band))];
+                    const int j = kt * KVT + jj;
+                    const double pj = 448.0 * exp2(s[jj] - m);
+                    l += pj;
+                    double pq = pj;
+                    uint8_t code = 0;
+                    if (!keep_p) {
+                        code = oracle_e4m3_encode(pj);
+                        pq = vdec[code];
+                    }
+                    for (int cc = 0; cc < D; cc++) {
+                        const double vv = keep_v ? (double)vph[(int64_t)j * D + cc] : vdec[vh[(int64_t)j * D + cc]];
+                        O[cc] += pq * vv;
+                    }
+                    if (unc && !keep_p) {
+                        const double band =
+                            2.0 * LN2 * U32 * (5.0 * mag[jj] + 7.0 * fabs(m) + 27.0) + EXP2_REL;
+                        const double lo = vdec[oracle_e4m3_encode(pj * (1.0 - band))];
+                        const double hi = vdec[oracle_e4m3_encode(pj * (1.0 + band))];
                         const double step = fmax(hi - pq, pq - lo);
                         if (step > 0)
-                            for (int cc = 0; cc < D; cc++) U[cc] += step * fabs(vdec[vrow[cc]]);
+                            for (int cc = 0; cc < D; cc++) {
+                                const double vv = keep_v ? (double)vph[(int64_t)j * D + cc] : vdec[vh[(int64_t)j * D + cc]];
+                                U[cc] += step * fabs(vv);
+                            }
                     }
                 }
             }
-            double *o = out + ((int64_t)t * QBLK + r) * D;
+            double *o = out + ((int64_t)t * QTILE + r) * D;
             const float *vs = v_scale + ((int64_t)b * p->Hkv + hk) * D;
             const float *mv = mean_v + ((int64_t)b * p->Hkv + hk) * D;
             for (int cc = 0; cc < D; cc++) {
-                o[cc] = O[cc] * (double)vs[cc] / l;
+                const double sc = keep_v ? 1.0 : (double)vs[cc];
+                o[cc] = O[cc] * sc / l;
                 if (p->smooth_v) o[cc] += (double)mv[cc];
-                if (unc) unc[((int64_t)t * QBLK + r) * D + cc] = U[cc] * (double)vs[cc] / l;
+                if (unc) unc[((int64_t)t * QTILE + r) * D + cc] = U[cc] * sc / l;
             }
             free(O);
             free(U);
             free(dS);
+            free(dmag);
         }
 }
 
@@ -471,9 +504,9 @@ void oracle_exact_attention_tiles(const oracle_params *p, const uint16_t *q, con
     const int D = p->D, Nq = p->Nq, Nkv = p->Nkv;
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int t = 0; t < n_tiles; t++)
-        for (int r = 0; r < QBLK; r++) {
+        for (int r = 0; r < QTILE; r++) {
             const int b = tiles[3 * t], h = tiles[3 * t + 1], qt = tiles[3 * t + 2];
-            const int i = qt * QBLK + r;
+            const int i = qt * QTILE + r;
             if (i >= Nq) continue;
             const int hk = h / (p->Hq / p->Hkv);
             double *qi = (double *)malloc(sizeof(double) * (size_t)D);
@@ -488,7 +521,7 @@ void oracle_exact_attention_tiles(const oracle_params *p, const uint16_t *q, con
                 if (s[j] > m) m = s[j];
             }
             double l = 0.0;
-            double *o = out + ((int64_t)t * QBLK + r) * D;
+            double *o = out + ((int64_t)t * QTILE + r) * D;
             for (int c = 0; c < D; c++) o[c] = 0.0;
             for (int j = 0; j < Nkv; j++) {
                 if (s[j] == -INFINITY) continue;

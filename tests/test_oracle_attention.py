@@ -11,11 +11,20 @@
   V gives the constant up to the FP8 rounding of P.
 - The fp64 exact attention equals PyTorch's scaled_dot_product_attention in
   fp64 (library routine), including causal masking and GQA.
+- With every quantisation step switched off (P, V and Q K^T unquantised) the
+  tiled online softmax is exact softmax attention: a dropped rescale, a wrong
+  running max, a masking or GQA index error would all show here.
+- Error decomposition on iid inputs: FP8 rounding of P alone and of V alone
+  each cost the closed-form rms relative error of e4m3 round-to-nearest
+  (2^-3/sqrt(12) * sqrt(3/(8 ln 2)) = 0.0265 for log-uniform mantissas), the
+  two together their quadrature sum, and INT8 Q K^T (per-token Q, 32-key K
+  scales) well below either.
+- The running max is the plain one: each tile's largest logit gets the FP8
+  code of 448 exactly and earlier tiles are rescaled by 2^(m_old - m_new).
 - The quantised mirror stays within the error the FP8/INT8 steps allow of the
-  exact result (relative L1 <= 0.06, cosine >= 0.998 on iid data: FP8 e4m3 has
-  a relative step of 2^-3, i.e. ~3.6% rms rounding error per operand; see the
-  measured values in the design notes), also when block scales differ by
-  orders of magnitude and when the running max grows tile after tile.
+  exact result (relative L1 <= 0.06, cosine >= 0.998 on iid data), also when
+  block scales differ by orders of magnitude and when the running max grows
+  tile after tile.
 """
 import numpy as np
 import pytest
@@ -200,17 +209,18 @@ def test_mirror_within_quantisation_error_of_exact(case):
 
 
 def test_mirror_uses_the_right_block_scales():
-    # K blocks (64 tokens) and Q blocks (128 tokens) with magnitudes that
-    # differ by orders of magnitude: a wrong block index in the scale lookup
-    # changes logits by large factors.
+    # K blocks (32 tokens) and Q tokens with magnitudes that differ by orders
+    # of magnitude: a wrong block or token index in the scale lookup changes
+    # logits by large factors.
     w = random_problem(1, 2, 2, 384, 384, 64, dtype="fp16", seed=12, k_offset_sigma=0.0)
     pr = _problem(w, smooth_k=False)
     q, k, v = generate(w)
     Q, K = oracle.to_double(pr, q), oracle.to_double(pr, k)
-    kscale = np.array([0.02, 1.0, 0.1, 3.0, 0.5, 0.05])
-    qscale = np.array([0.1, 2.0, 0.5])
-    K = K * np.repeat(kscale, 64)[None, None, :, None]
-    Q = Q * np.repeat(qscale, 128)[None, None, :, None]
+    rng = np.random.default_rng(3)
+    kscale = 10.0 ** rng.uniform(-1.5, 0.5, 384 // 32)
+    qscale = 10.0 ** rng.uniform(-1.0, 0.3, 384)
+    K = K * np.repeat(kscale, 32)[None, None, :, None]
+    Q = Q * qscale[None, None, :, None]
     q = Q.astype(np.float16).view(np.uint16)
     k = K.astype(np.float16).view(np.uint16)
     pre = oracle.prepass(pr, q, k, v)
@@ -258,11 +268,110 @@ def test_uncertainty_is_zero_when_p_codes_are_exact_and_small_otherwise():
     pre = oracle.prepass(pr, np.zeros_like(q), k, v)
     _, unc = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr), with_uncertainty=True)
     assert np.all(unc == 0)
-    # random inputs: a few ambiguous codes, each worth at most one e4m3 step
+    # random inputs: a few ambiguous codes (a fraction of the outputs sees
+    # one of its 300 keys ambiguous), each worth at most one e4m3 step
     pre = oracle.prepass(pr, q, k, v)
     out, unc = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr), with_uncertainty=True)
     assert np.all(unc >= 0)
-    assert 0 < (unc > 0).mean() < 0.05
-    assert unc.max() < 0.05 * np.abs(out).max()
+    assert 0 < (unc > 0).mean() < 0.25
+    assert unc.max() < 0.01 * np.abs(out).max()
+    assert unc.mean() < 1e-3 * np.abs(out).mean()
     # the mirror itself is unchanged by asking for the bound
     assert np.array_equal(out, oracle.attention_tiles(pr, pre, oracle.all_tiles(pr)))
+
+
+ALL_EXACT = oracle.KEEP_P | oracle.KEEP_V | oracle.KEEP_QK
+
+EXACT_CASES = [
+    dict(args=(1, 2, 2, 256, 256, 64), dtype="fp16"),
+    dict(args=(2, 4, 2, 300, 520, 96), dtype="bf16", layout="NHD"),
+    dict(args=(1, 4, 1, 384, 384, 128), dtype="bf16", is_causal=True),
+    dict(args=(1, 2, 2, 200, 700, 64), dtype="fp16", is_causal=True),
+    dict(args=(1, 2, 2, 256, 512, 128), dtype="fp16", smooth_q=True, smooth_v=True),
+    dict(args=(1, 2, 1, 129, 300, 64), dtype="bf16", smooth_k=False, smooth_v=True),
+]
+
+
+@pytest.mark.parametrize("case", EXACT_CASES, ids=[str(i) for i in range(len(EXACT_CASES))])
+def test_mirror_with_nothing_quantised_is_exact_attention(case):
+    flags = {k: v for k, v in case.items() if k in ("is_causal", "smooth_k", "smooth_q", "smooth_v")}
+    w = random_problem(*case["args"], layout=case.get("layout", "HND"), dtype=case["dtype"], seed=17,
+                       k_offset_sigma=3.0)
+    pr = _problem(w, **flags)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v, keep_fp32=True)
+    t = oracle.all_tiles(pr)
+    m = oracle.attention_tiles(pr, pre, t, exact_mask=ALL_EXACT)
+    e = oracle.exact_attention_tiles(pr, q, k, v, t)
+    rows = np.zeros((len(t), 128), bool)
+    for n, (_, _, qt) in enumerate(t):
+        rows[n, : max(0, min(128, pr.Nq - 128 * qt))] = True
+    # only the fp32 rounding of the smoothed inputs (Q - mq, K - mean_k,
+    # V - mean_v) separates the two
+    assert np.max(np.abs(m[rows] - e[rows])) <= 1e-5 * np.max(np.abs(e[rows]))
+    # quantising anything moves it by far more than that
+    assert np.max(np.abs(oracle.attention_tiles(pr, pre, t)[rows] - e[rows])) > 1e-3
+
+
+# rms relative error of e4m3 round-to-nearest for log-uniform mantissas:
+# step 2^-3 relative to the binade start, error uniform in half a step,
+# E[2^-2u] = 3 / (8 ln 2) over u ~ U(0, 1)
+E4M3_RMS = 2.0 ** -3 / np.sqrt(12.0) * np.sqrt(3.0 / (8.0 * np.log(2.0)))
+
+
+def test_error_decomposition_iid():
+    w = random_problem(1, 2, 2, 768, 1024, 128, dtype="bf16", seed=18, k_offset_sigma=3.0)
+    pr = _problem(w)
+    q, k, v = generate(w)
+    pre = oracle.prepass(pr, q, k, v, keep_fp32=True)
+    t = oracle.all_tiles(pr)
+    e = oracle.exact_attention_tiles(pr, q, k, v, t)
+    err = {}
+    for name, keep in dict(p=ALL_EXACT ^ oracle.KEEP_P, v=ALL_EXACT ^ oracle.KEEP_V,
+                           qk=ALL_EXACT ^ oracle.KEEP_QK, pv=oracle.KEEP_QK, all=0).items():
+        err[name] = _rel_l1(oracle.attention_tiles(pr, pre, t, exact_mask=keep), e)
+    # FP8 P and FP8 V alone: the e4m3 rms error (P a little less: each row's
+    # maximum gets the exact code 448)
+    assert 0.80 * E4M3_RMS <= err["p"] <= 1.05 * E4M3_RMS, err
+    assert 0.90 * E4M3_RMS <= err["v"] <= 1.10 * E4M3_RMS, err
+    # independent roundings add in quadrature
+    assert abs(err["pv"] - np.hypot(err["p"], err["v"])) <= 0.08 * err["pv"], err
+    # INT8 Q K^T with per-token Q and 32-key K scales is the small part
+    assert err["qk"] <= 0.5 * err["p"], err
+    total = np.sqrt(err["p"] ** 2 + err["v"] ** 2 + err["qk"] ** 2)
+    assert abs(err["all"] - total) <= 0.10 * total, err
+    assert err["all"] <= 0.045, err
+
+
+def test_running_max_is_the_plain_one():
+    # One query row, two KV tiles.  The largest logit of tile 1 sits at key
+    # j1, that of tile 2 at key j2 with s(j2) - s(j1) = d in (0, 1).  V is an
+    # indicator: channel 0 of key j2, channel 1 of key j1 (both decode to
+    # exactly 1).  With the plain running max each tile's largest logit gets
+    # P code 448 and tile 1's contribution is rescaled by 2^-d when tile 2
+    # raises the max, so o_1 / o_0 = 2^(s(j1) - s(j2)) exactly; a max raised
+    # only past a threshold would leave tile 1 unscaled and give key j2 a code
+    # other than 448.
+    D, Nkv = 64, 256
+    w = random_problem(1, 1, 1, 1, Nkv, D, dtype="fp16", seed=19, k_offset_sigma=0.0)
+    pr = _problem(w, smooth_k=False)
+    qv = np.zeros((1, 1, 1, D))
+    qv[0, 0, 0, 0] = 1.0
+    kv = np.zeros((1, 1, Nkv, D))
+    kv[0, 0, :, 0] = np.linspace(-2.0, 1.0, Nkv)       # logits rise with j
+    j1, j2 = 100, 200
+    kv[0, 0, j1, 0] = 2.0                                # tile 1's maximum
+    kv[0, 0, j2, 0] = 2.5                                # tile 2's, higher by less than 1 in log2
+    kv[0, 0, :, 1] = 1.0                                 # keep every K block's amax equal
+    vv = np.zeros((1, 1, Nkv, D))
+    vv[0, 0, j2, 0] = 1.0
+    vv[0, 0, j1, 1] = 1.0
+    q, k, v = (x.astype(np.float16).view(np.uint16) for x in (qv, kv, vv))
+    pre = oracle.prepass(pr, q, k, v)
+    o = oracle.attention_tiles(pr, pre, oracle.all_tiles(pr))[0, 0]
+    S = pre["k8"][0, 0].astype(np.int64) @ pre["q8"][0, 0, 0].astype(np.int64)
+    c = (pre["q_scale"][0, 0, 0].astype(np.float64) * pre["k_scale"][0, 0].astype(np.float64)
+         * float(pr.resolved_sm_scale()) / np.log(2.0))
+    s = S * np.repeat(c, 32)
+    assert np.argmax(s[:128]) == j1 and np.argmax(s) == j2 and 0 < s[j2] - s[j1] < 1
+    assert abs(o[1] / o[0] - 2.0 ** (s[j1] - s[j2])) <= 1e-12

@@ -58,11 +58,14 @@ def test_k_prime_is_k_minus_mean(case):
 
 
 def _check_int8_blocks(x, codes, scales, blk, axis_len):
+    """Blocks of `blk` tokens (all D channels) along axis -2, one scale each."""
     nb = (axis_len + blk - 1) // blk
     assert scales.shape[-1] == nb
     for i in range(nb):
         sl = slice(i * blk, min((i + 1) * blk, axis_len))
         xb, cb, s = x[..., sl, :], codes[..., sl, :].astype(np.float64), scales[..., i]
+        if not np.any(s):
+            continue
         amax = np.abs(xb).max(axis=(-2, -1))
         assert np.array_equal(s, (amax.astype(np.float32) / np.float32(127)))
         assert np.all(np.abs(cb) <= 127)
@@ -72,37 +75,40 @@ def _check_int8_blocks(x, codes, scales, blk, axis_len):
         assert np.all(err <= s[..., None, None] * (0.5 + 2.0 ** -16))
 
 
-def test_k_int8_blocks_of_64(case):
+def test_k_int8_blocks_of_32(case):
     pr, q, k, v, pre = case
-    _check_int8_blocks(pre["kp"].astype(np.float64), pre["k8"], pre["k_scale"], 64, pr.Nkv)
+    assert pre["k_scale"].shape[-1] == (pr.Nkv + 31) // 32
+    _check_int8_blocks(pre["kp"].astype(np.float64), pre["k8"], pre["k_scale"], 32, pr.Nkv)
 
 
-def test_q_int8_blocks_of_128_with_smoothing(case):
+def test_q_int8_per_token_with_block_mean_smoothing(case):
     pr, q, k, v, pre = case
     Q = _hnd(pr, q, pr.Hq, pr.Nq)
-    nqb = pr.nqb
     qp = np.empty_like(Q)
-    for i in range(nqb):
+    for i in range(pr.nmb):
         sl = slice(i * 128, min((i + 1) * 128, pr.Nq))
         mean = Q[:, :, sl].mean(axis=2)
         assert np.all(np.abs(pre["mq"][:, :, i] - mean) <= 2.0 ** -25 + np.abs(mean) * 2.0 ** -23)
         qp[:, :, sl] = (Q[:, :, sl].astype(np.float32) - pre["mq"][:, :, i][:, :, None, :])
-    _check_int8_blocks(qp, pre["q8"], pre["q_scale"], 128, pr.Nq)
+    assert pre["q_scale"].shape == (pr.B, pr.Hq, pr.Nq)
+    _check_int8_blocks(qp, pre["q8"], pre["q_scale"], 1, pr.Nq)
+    # the fp32 Q' the pre-pass hands to the error decomposition is the same
+    pre32 = oracle.prepass(pr, q, k, v, keep_fp32=True)
+    assert np.array_equal(pre32["qp"].astype(np.float64), qp)
 
 
 def test_ragged_last_block_uses_only_valid_tokens():
-    # Last K block has 8 tokens; a huge value planted in the tokens *after* Nkv
-    # (i.e. not part of the input) cannot exist, so instead check the ragged
-    # block's scale equals the amax of its own 8 tokens only.
+    # The last K block has 8 tokens: its scale is the amax of those 8 only;
+    # the last Q token's scale is its own amax.
     w = random_problem(1, 1, 1, 130, 72, 64, seed=9, k_offset_sigma=0.0)
     pr = _problem(w, smooth_k=False)
     q, k, v = generate(w)
     pre = oracle.prepass(pr, q, k, v)
     K = _hnd(pr, k, 1, 72)
-    assert pre["k_scale"].shape[-1] == 2
-    assert pre["k_scale"][0, 0, 1] == np.float32(np.abs(K[0, 0, 64:72]).max()) / np.float32(127)
+    assert pre["k_scale"].shape[-1] == 3
+    assert pre["k_scale"][0, 0, 2] == np.float32(np.abs(K[0, 0, 64:72]).max()) / np.float32(127)
     Q = _hnd(pr, q, 1, 130)
-    assert pre["q_scale"][0, 0, 1] == np.float32(np.abs(Q[0, 0, 128:130]).max()) / np.float32(127)
+    assert pre["q_scale"][0, 0, 129] == np.float32(np.abs(Q[0, 0, 129]).max()) / np.float32(127)
 
 
 def test_zero_block_has_zero_scale_and_codes():
@@ -110,11 +116,15 @@ def test_zero_block_has_zero_scale_and_codes():
     pr = _problem(w, smooth_k=False)
     q, k, v = generate(w)
     k = k.copy()
-    k[0, 0, 64:128] = 0  # second K block all zero (fp16 +0 bits)
+    k[0, 0, 64:96] = 0   # third K block all zero (fp16 +0 bits)
+    q = q.copy()
+    q[0, 0, 5] = 0       # query token 5 all zero
     v = v.copy()
     v[0, 0, :, 3] = 0    # channel 3 of V all zero
     pre = oracle.prepass(pr, q, k, v)
-    assert pre["k_scale"][0, 0, 1] == 0 and np.all(pre["k8"][0, 0, 64:] == 0)
+    assert pre["k_scale"][0, 0, 2] == 0 and np.all(pre["k8"][0, 0, 64:96] == 0)
+    assert pre["k_scale"][0, 0, 1] > 0 and pre["k_scale"][0, 0, 3] > 0
+    assert pre["q_scale"][0, 0, 5] == 0 and np.all(pre["q8"][0, 0, 5] == 0)
     assert pre["v_scale"][0, 0, 3] == 0 and np.all(pre["v8"][0, 0, :, 3] == 0)
 
 
