@@ -4,7 +4,8 @@
 
 A step is one whole pass (smoothing + quantisation pre-pass, then the
 attention kernel) over one batch of the named synthetic workload (default:
-B4 H32 N4096 D128 bf16 HND, non-causal), inputs resident in HBM.  The metric
+causal GQA prefill B1 Hq32 Hkv8 N32768 D128 bf16, the N >= 8K, d = 128 case
+the throughput target is stated for), inputs resident in HBM.  The metric
 is attention TOPS = 4*B*Hq*Nq*Nkv*D / time (halved for causal), whole job.
 Under torchrun (N > 1) every rank runs the same workload on its own GPU
 (independent replicas, no collective in the data path: the pass does not
@@ -12,9 +13,10 @@ shard across GPUs); the time is the max over ranks.
 
 Reported beside the value: the attention kernel's roofline (tensor-bound,
 8-bit peak derived from the measured bf16 GEMM peak x 2, the nominal 8-bit /
-16-bit ratio), the end-to-end number through the public API with host
-buffers, SM clocks sampled during the timed region, and the CPU oracle timed
-on a bounded sample (``cpu_baseline``).  ``--impl reference`` times the CPU
+16-bit ratio, and beside it the rate of back-to-back tcgen05 8-bit MMAs
+measured in the same run), the end-to-end number through the public API with
+host buffers, SM clocks sampled during the timed region, and the CPU oracle
+timed on a bounded sample (``cpu_baseline``).  ``--impl reference`` times the CPU
 oracle itself on the same workload, one bounded sample per step.
 """
 from __future__ import annotations
@@ -36,14 +38,14 @@ sys.path.insert(0, ROOT)
 from quantized_attention_subtract_b200.workloads import WORKLOADS, Workload, generate  # noqa: E402
 
 METRIC = "attention TOPS (4*B*H*Nq*Nkv*d/s) at N=4K-32K, d=128; % of B200 tensor peak"
-DEFAULT_WORKLOAD = "mha_n4096_d128_bf16"
+DEFAULT_WORKLOAD = "gqa_causal_n32768_d128_bf16"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM bytes (read + write) per launch of the attention kernel on the default
-# workload, from one ncu capture (profiles/attn_fwd_kernel_mha_n4096_d128_bf16.md).
-# They describe the kernel built from the sources hashed here; after any change
-# to those sources the traffic is reported as null until it is captured again.
-ATTN_TRAFFIC = {"workload": DEFAULT_WORKLOAD, "sources_sha256_16": "398152f62f5a2346", "bytes": 300471040}
+# DRAM bytes (read + write) per launch of the attention kernel, from one ncu
+# capture per workload.  They describe the kernel built from the sources hashed
+# here; after any change to those sources the traffic is reported as null until
+# it is captured again.
+ATTN_TRAFFIC = {}   # workload name -> {"sources_sha256_16": ..., "bytes": ...}
 ATTN_SOURCES = ["attn_fwd.cu", "ptx.cuh", "common.cuh"]
 
 
@@ -61,11 +63,10 @@ def _attn_traffic(w: Workload):
         data = b"".join(open(os.path.join(csrc, f), "rb").read() for f in ATTN_SOURCES)
     except OSError:
         return None
-    if w.name != ATTN_TRAFFIC["workload"]:
+    rec = ATTN_TRAFFIC.get(w.name)
+    if rec is None or hashlib.sha256(data).hexdigest()[:16] != rec["sources_sha256_16"]:
         return None
-    if hashlib.sha256(data).hexdigest()[:16] != ATTN_TRAFFIC["sources_sha256_16"]:
-        return None
-    return ATTN_TRAFFIC["bytes"]
+    return rec["bytes"]
 
 
 def _peaks():
@@ -75,6 +76,28 @@ def _peaks():
         return float(m["bf16_tflops"]), float(m["hbm_gbs"]), "measured"
     except Exception:
         return 1590.0, 6650.0, "fallback"
+
+
+def mma_loop_peak(dev, iters: int = 4096):
+    """TOPS of back-to-back tcgen05 8-bit MMAs (128x256x32, operands resident
+    in shared memory) on one CTA per SM, INT8 and FP8 kinds, timed with CUDA
+    events after a warm-up: the attainable 8-bit tensor rate of this GPU."""
+    import torch
+    from quantized_attention_subtract_b200 import binding
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    sink = torch.zeros(sms + 1, dtype=torch.int32, device=dev)
+    out = {}
+    for kind, name in ((0, "i8"), (1, "e4m3")):
+        binding.debug_mma_loop(sms, 256, sink, kind)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        binding.debug_mma_loop(sms, iters, sink, kind)
+        b.record()
+        torch.cuda.synchronize(dev)
+        assert int(sink[sms]) == 0, "MMA loop status"
+        ops = 2.0 * 128 * 256 * 128 * iters * sms   # 4 MMAs of K=32 per iteration
+        out[name] = ops / (a.elapsed_time(b) * 1e-3) / 1e12
+    return out
 
 
 def _dist():
@@ -331,6 +354,7 @@ def run_ours(args, w: Workload):
     peak8 = 2.0 * bf16_tflops  # 8-bit dense = 2 x bf16 dense (nominal 4.5 / 2.25 PFLOP/s)
     achieved = w.ops / (attn_ms * 1e-3) / 1e12
     value = replica_value(world, w.ops, step_ms)
+    mma_peak = mma_loop_peak(dev)
     kernels_per_step = 4 + (1 if w.smooth_q else 0)  # kv_stats, kv_finalize, quantize, (delta_s), attention
 
     line = {
@@ -344,8 +368,10 @@ def run_ours(args, w: Workload):
                    "l2": f"inputs {in_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)"},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
                      "peak": peak8, "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": _attn_traffic(w),
-                     "peak_source": f"{peak_src} bf16 x 2 (burst)", "attn_ms": attn_ms,
-                     "prepass_ms": pre_ms,
+                     "peak_source": f"{peak_src} bf16 x 2 (burst)",
+                     "peak_measured_mma_loop": mma_peak,
+                     "frac_of_mma_loop_i8": achieved / mma_peak["i8"],
+                     "attn_ms": attn_ms, "prepass_ms": pre_ms,
                      "prepass_gbs": _prepass_bytes(w, qd, kd, vd) / (pre_ms * 1e-3) / 1e9},
         "e2e": {"value": replica_value(world, w.ops, e2e_ms), "unit": "TOPS",
                 "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": out.numel() * 2},

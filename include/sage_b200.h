@@ -12,14 +12,15 @@
  *   1. smoothing: subtract the per-channel mean of K over all tokens
  *      (smooth_k); optionally subtract per-block Q means (smooth_q) and V
  *      channel means (smooth_v), with their exact correction terms;
- *   2. quantisation: per-block symmetric INT8 Q (128 tokens) and K (64
- *      tokens) with fp32 scales; V to FP8 e4m3 with per-channel scales;
+ *   2. quantisation: symmetric INT8 Q with one fp32 scale per token and K
+ *      with one per block of 32 tokens (the pages' per-block / per-thread
+ *      granularity: closerAI blog, part 4; "SageAttention2: Technical
+ *      report", section 1); V to FP8 e4m3 with per-channel scales;
  *   3. a flash-style kernel: INT8 Q K^T with exact int32 accumulation,
- *      dequantisation, online softmax (running max and sum, exp2), P
- *      quantised to FP8 e4m3 as 224 * exp2(s - m), where m is a per-row
- *      reference max raised to a tile's max only when that exceeds m by more
- *      than 1 (so every value stays within e4m3's 448), FP8 P V with fp32
- *      accumulation;
+ *      dequantisation, online softmax in base 2 with the row's running max
+ *      m raised to every 128-key tile's max and the running sum rescaled
+ *      with it, P quantised to FP8 e4m3 as 448 * exp2(s - m) (at most 448,
+ *      e4m3's largest finite value), FP8 P V with fp32 accumulation;
  *   4. epilogue: divide by the row sum, rescale by the V channel scale (and
  *      add the V mean back), round to the input's 16-bit type.
  *
@@ -50,7 +51,7 @@
 extern "C" {
 #endif
 
-#define SAGE_ABI_VERSION 3
+#define SAGE_ABI_VERSION 4
 
 /* A CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st *sage_stream_t;
@@ -89,10 +90,6 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
  * comes from sage_workspace_size() and it must be 256-byte aligned.
  * Precondition of the exact fixed-point means: |x| * N < 2^39 for every
  * smoothed input x (e.g. |x| < 2^24 at N = 32768).  Inputs must be finite.
- * fuse_q = 1 asks the whole pass (sage_attn_fwd and its two halves) to
- * quantise Q inside the attention kernel instead of in the pre-pass; it
- * applies without smooth_q and when the driver accepts a tensor map of q's
- * strides, and gives the same q8, q_scale and output bit for bit.
  */
 typedef struct {
   const void *q, *k, *v;
@@ -102,7 +99,6 @@ typedef struct {
   int32_t layout;               /* sage_layout_t */
   int32_t dtype;                /* sage_dtype_t */
   int32_t is_causal, smooth_k, smooth_q, smooth_v;
-  int32_t fuse_q;               /* 0 or 1, see below */
   float sm_scale;
   void *workspace;
   size_t workspace_bytes;
@@ -115,7 +111,7 @@ typedef struct {
    * (they size the workspace); a sequence with queries needs at least one
    * key.  Each sequence is its own problem (its own smoothing means and V
    * scales; causal masking top-left within it).  The arrays are copied
-   * during the call.  fuse_q has no effect here. */
+   * during the call. */
   const int32_t *cu_seqlens_q, *cu_seqlens_kv;
 } sage_attn_params_t;
 
@@ -127,8 +123,8 @@ typedef struct {
   int8_t *q8;        /* [B*Hq ][Nq_pad ][Dp]  INT8 codes of Q (or Q - mq)       */
   int8_t *k8;        /* [B*Hkv][Nkv_pad][Dp]  INT8 codes of K - mean_k           */
   uint8_t *v8t;      /* [B*Hkv][D][Nkv_pad]   FP8 e4m3 codes of V (- mean_v), transposed */
-  float *q_scale;    /* [B*Hq ][Nq_pad/128]                                      */
-  float *k_scale;    /* [B*Hkv][Nkv_pad/64]                                      */
+  float *q_scale;    /* [B*Hq ][Nq_pad]       one per query token (0 past Nq)    */
+  float *k_scale;    /* [B*Hkv][Nkv_pad/32]   one per 32 keys                    */
   float *v_scale;    /* [B*Hkv][D]                                               */
   float *mean_k;     /* [B*Hkv][D]   (zeros when smooth_k == 0)                  */
   float *mean_v;     /* [B*Hkv][D]   (zeros when smooth_v == 0)                  */
@@ -154,19 +150,15 @@ sage_status_t sage_workspace_view(const sage_attn_params_t *p, sage_workspace_vi
 
 /* The whole pass: smoothing + quantisation pre-pass, then the attention
  * kernel, enqueued on `stream`.  Writes p->out.  Also resets the device
- * status word at its start.  With fuse_q (see sage_attn_params_t) Q is
- * quantised by the attention kernel (same codes and scale as the pre-pass
- * would give; they are written to the workspace too). */
+ * status word at its start. */
 sage_status_t sage_attn_fwd(const sage_attn_params_t *p, sage_stream_t stream);
 
 /* The two halves of sage_attn_fwd, exposed so that their device time can be
  * measured apart; calling sage_attn_fwd_prepass and then
  * sage_attn_fwd_attention with the same parameters and workspace is
- * equivalent to sage_attn_fwd.  With fuse_q in effect the attention half
- * quantises Q itself (from p->q, to the workspace's q8 / q_scale as well) and
- * the pre-pass half quantises only K and V; otherwise the pre-pass half is
- * sage_quantize and the attention half sage_attn_quantized.  The pre-pass
- * half resets the device status word.  Errors as for sage_attn_fwd. */
+ * equivalent to sage_attn_fwd (they are sage_quantize and
+ * sage_attn_quantized).  The pre-pass half resets the device status word.
+ * Errors as for sage_attn_fwd. */
 sage_status_t sage_attn_fwd_prepass(const sage_attn_params_t *p, sage_stream_t stream);
 sage_status_t sage_attn_fwd_attention(const sage_attn_params_t *p, sage_stream_t stream);
 
@@ -195,15 +187,24 @@ sage_status_t sage_attn_quantized(const sage_attn_params_t *p, sage_stream_t str
  * contents; each call clears what must start at zero.  Calls that overlap on
  * the GPU (other streams, other threads) race on the array and must be
  * serialised by the caller.  sage_get_device_status does not see this
- * array; a device timeout still makes later results unreliable.
+ * array; read it with sage_noalloc_device_status.
  * The SageAttention pages have no counterpart of this call. */
 #define SAGE_NOALLOC_MAX_WORKSPACE_BYTES (64ull << 20)
 sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t stream);
 
-/* Debug: the int32 tile S = q8 k8^T of query tile `qtile` (128 rows) and key
- * tile `ktile` (128 keys) of (batch b, query head h), computed by the same
- * tensor-core path as the attention kernel from a filled workspace, written
- * row-major to the device buffer s_out[128*128]. */
+/* Synchronously read the device status word that the last
+ * sage_attn_fwd_noalloc call with the same shapes and flags left in the
+ * library scratch of the current device (SAGE_OK when no kernel recorded a
+ * failure).  p's workspace fields are ignored.  No counterpart on the pages. */
+sage_status_t sage_noalloc_device_status(const sage_attn_params_t *p, int32_t *code);
+
+/* Debug: the attention half of the pass (as sage_attn_quantized, on a
+ * workspace that sage_quantize filled; it writes p->out too) in a build of
+ * the attention kernel that also copies the int32 tile S = q8 k8^T of query
+ * tile `qtile` (128 rows) and key tile `ktile` (128 keys) of (batch b, query
+ * head h), as its softmax warps read it from tensor memory, row-major to the
+ * device buffer s_out[128*128].  Key tiles a causal query tile skips are not
+ * computed (s_out is then left untouched).  Not for variable-length batches. */
 sage_status_t sage_debug_dump_s(const sage_attn_params_t *p, int32_t b, int32_t h, int32_t qtile,
                                 int32_t ktile, int32_t *s_out, sage_stream_t stream);
 
@@ -219,11 +220,17 @@ sage_status_t sage_debug_pv(const sage_attn_params_t *p, int32_t b, int32_t hkv,
  * order (element 2i in the low byte of each packed pair). */
 sage_status_t sage_debug_e4m3(const float *in, uint8_t *out, int64_t n, sage_stream_t stream);
 
-/* Debug: back-to-back INT8 tensor-core MMAs (128x256x32 each, operands
- * resident in shared memory) on `ctas` CTAs for `iters` iterations; used to
- * measure the attainable 8-bit MMA rate.  `sink` is a device int32 buffer of
- * ctas + 1 entries: one value per CTA, then a status word the waits use. */
-sage_status_t sage_debug_mma_loop(int32_t ctas, int32_t iters, int32_t *sink, sage_stream_t stream);
+/* Debug: back-to-back 8-bit tensor-core MMAs (128x256x32 each, operands
+ * resident in shared memory; kind 0 = INT8 -> S32, kind 1 = FP8 e4m3 -> F32)
+ * on `ctas` CTAs for `iters` iterations; used to measure the attainable
+ * 8-bit MMA rate.  `sink` is a device int32 buffer of ctas + 1 entries: one
+ * value per CTA, then a status word the waits use. */
+sage_status_t sage_debug_mma_loop(int32_t ctas, int32_t iters, int32_t kind, int32_t *sink,
+                                  sage_stream_t stream);
+
+/* Debug: the attention kernel's exp2 (the hardware ex2.approx.ftz.f32)
+ * applied to n device floats; used to measure its error against fp64. */
+sage_status_t sage_debug_ex2(const float *in, float *out, int64_t n, sage_stream_t stream);
 
 /* Debug: one thread waits on a shared-memory barrier that nothing completes,
  * through the same bounded wait every kernel uses; after about one second the

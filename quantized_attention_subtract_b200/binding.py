@@ -25,9 +25,11 @@ STATUS_NAMES = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTE
 # Every symbol include/sage_b200.h declares.
 EXPORTED = ["sage_abi_version", "sage_status_string", "sage_workspace_size", "sage_workspace_view",
             "sage_attn_fwd", "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
-            "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop", "sage_debug_wait_timeout",
-            "sage_get_device_status", "sage_attn_fwd_noalloc", "sage_attn_fwd_prepass",
-            "sage_attn_fwd_attention"]
+            "sage_debug_pv", "sage_debug_e4m3", "sage_debug_ex2", "sage_debug_mma_loop",
+            "sage_debug_wait_timeout", "sage_get_device_status", "sage_attn_fwd_noalloc",
+            "sage_noalloc_device_status", "sage_attn_fwd_prepass", "sage_attn_fwd_attention"]
+
+ABI_VERSION = 4
 
 
 class SageError(RuntimeError):
@@ -48,7 +50,7 @@ class Params(ctypes.Structure):
         ("layout", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("is_causal", ctypes.c_int32), ("smooth_k", ctypes.c_int32),
         ("smooth_q", ctypes.c_int32), ("smooth_v", ctypes.c_int32),
-        ("fuse_q", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+        ("sm_scale", ctypes.c_float),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_kv", ctypes.c_void_p),
     ]
@@ -88,15 +90,21 @@ def lib():
             L.sage_debug_dump_s.argtypes = [P, i32, i32, i32, i32, vp, vp]
             L.sage_debug_pv.argtypes = [P, i32, i32, i32, vp, vp, vp]
             L.sage_debug_e4m3.argtypes = [vp, vp, ctypes.c_int64, vp]
-            L.sage_debug_mma_loop.argtypes = [i32, i32, vp, vp]
+            L.sage_debug_ex2.argtypes = [vp, vp, ctypes.c_int64, vp]
+            L.sage_debug_mma_loop.argtypes = [i32, i32, i32, vp, vp]
             L.sage_get_device_status.argtypes = [P, ctypes.POINTER(i32)]
+            L.sage_noalloc_device_status.argtypes = [P, ctypes.POINTER(i32)]
             L.sage_debug_wait_timeout.argtypes = [vp, vp]
             for name in ("sage_workspace_size", "sage_workspace_view", "sage_attn_fwd",
                          "sage_quantize", "sage_attn_quantized", "sage_debug_dump_s",
-                         "sage_debug_pv", "sage_debug_e4m3", "sage_debug_mma_loop",
+                         "sage_debug_pv", "sage_debug_e4m3", "sage_debug_ex2", "sage_debug_mma_loop",
                          "sage_debug_wait_timeout", "sage_get_device_status",
-                         "sage_attn_fwd_noalloc"):
+                         "sage_attn_fwd_noalloc", "sage_noalloc_device_status",
+                         "sage_attn_fwd_prepass", "sage_attn_fwd_attention"):
                 getattr(L, name).restype = ctypes.c_int
+            if L.sage_abi_version() != ABI_VERSION:
+                raise RuntimeError(f"{LIB_PATH} has ABI version {L.sage_abi_version()}, "
+                                   f"this binding expects {ABI_VERSION}: rebuild it")
             _lib = L
     return _lib
 
@@ -108,6 +116,13 @@ def _check(code: int, what: str):
 
 def _stream(device: torch.device | None = None) -> ctypes.c_void_p:
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _call(name: str, p, device) -> None:
+    """Run entry point `name` on params p and the current stream of `device`,
+    with that device current (the library works on the current device)."""
+    with torch.cuda.device(device):
+        _check(getattr(lib(), name)(ctypes.byref(p), _stream(device)), name)
 
 
 def _dims(x: torch.Tensor, layout: str):
@@ -123,7 +138,7 @@ def _dims(x: torch.Tensor, layout: str):
 
 
 def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scale=None,
-                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None, fuse_q=False) -> Params:
+                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None) -> Params:
     """Fill sage_attn_params_t from torch tensors (no copies, strides as given)."""
     B, Hq, Nq, D = _dims(q, tensor_layout)
     Bk, Hkv, Nkv, Dk = _dims(k, tensor_layout)
@@ -144,7 +159,6 @@ def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scal
     p.dtype = 0 if q.dtype == torch.float16 else 1
     p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
                                                        int(bool(smooth_q)), int(bool(smooth_v)))
-    p.fuse_q = int(bool(fuse_q))
     p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
     if workspace is not None:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
@@ -192,7 +206,6 @@ def make_varlen_params(q, k, v, out, cu_seqlens_q, cu_seqlens_kv, max_seqlen_q=N
     p.dtype = 0 if q.dtype == torch.float16 else 1
     p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
                                                        int(bool(smooth_q)), int(bool(smooth_v)))
-    p.fuse_q = 0
     p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
     p.cu_seqlens_q, p.cu_seqlens_kv = cq.ctypes.data, ck.ctypes.data
     p._offsets = (cq, ck)  # the arrays must outlive every call made with p
@@ -239,7 +252,7 @@ def alloc_workspace(p: Params, device) -> torch.Tensor:
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
              is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
              smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
-             workspace: torch.Tensor | None = None, fuse_q: bool = False) -> torch.Tensor:
+             workspace: torch.Tensor | None = None) -> torch.Tensor:
     """Quantized attention forward: INT8 Q K^T, FP8 P V, on the current CUDA stream.
 
     q: [B, Hq, Nq, D] ("HND") or [B, Nq, Hq, D] ("NHD"); k, v: same with Hkv, Nkv.
@@ -248,22 +261,21 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
     copy of one chunk, the kernels of the previous one and the device-to-host
     copy of the one before overlap; the returned host tensor is complete once
     the current stream has passed this call (pinned host tensors make the
-    copies asynchronous).  fuse_q: quantise Q inside the attention kernel
-    instead of in the pre-pass (no effect with smooth_q; same results).
+    copies asynchronous).
     """
     if not q.is_cuda:
         return _sageattn_host(q, k, v, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                              smooth_v, out, fuse_q)
+                              smooth_v, out)
     if not (k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be on the same device")
     dev_out = torch.empty_like(q) if out is None else out
     p = make_params(q, k, v, dev_out, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                    smooth_v, fuse_q=fuse_q)
+                    smooth_v)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     else:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
-    _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(q.device)), "sage_attn_fwd")
+    _call("sage_attn_fwd", p, q.device)
     return dev_out
 
 
@@ -291,8 +303,7 @@ def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int, layout: s
     return chunks
 
 
-def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out,
-                   fuse_q=False):
+def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out):
     dev = torch.device("cuda", torch.cuda.current_device())
     B, Hq, Nq, D = _dims(q, layout)
     _, Hkv, Nkv, _ = _dims(k, layout)
@@ -316,7 +327,7 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
     first = make_params(sl(qd, *chunks[0][:1], chunks[0][1] * group, chunks[0][2] * group),
                         sl(kd, *chunks[0]), sl(vd, *chunks[0]),
                         sl(od, chunks[0][0], chunks[0][1] * group, chunks[0][2] * group),
-                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, fuse_q=fuse_q)
+                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
     ws = alloc_workspace(first, dev)
     done_out = None
     for b, h0, h1 in chunks:
@@ -330,13 +341,12 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
             landed = torch.cuda.Event()
             landed.record(h2d)
         compute.wait_event(landed)
-        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v,
-                        fuse_q=fuse_q)
+        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
         need = workspace_bytes(p)
         if need > ws.numel():
             ws = torch.empty(need, dtype=torch.uint8, device=dev)
         p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
-        _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(dev)), "sage_attn_fwd")
+        _call("sage_attn_fwd", p, dev)
         computed = torch.cuda.Event()
         computed.record(compute)
         d2h.wait_event(computed)
@@ -358,27 +368,36 @@ def attn_fwd_noalloc(p: Params, device) -> None:
     """sage_attn_fwd on the library's own static scratch (p.workspace is
     ignored); for callers that cannot allocate device memory on the call path.
     Calls share that scratch: serialise them."""
-    _check(lib().sage_attn_fwd_noalloc(ctypes.byref(p), _stream(device)), "sage_attn_fwd_noalloc")
+    _call("sage_attn_fwd_noalloc", p, device)
+
+
+def noalloc_device_status(p: Params, device) -> int:
+    """Device status word the last attn_fwd_noalloc call with p's shapes left."""
+    code = ctypes.c_int32(0)
+    with torch.cuda.device(device):
+        _check(lib().sage_noalloc_device_status(ctypes.byref(p), ctypes.byref(code)),
+               "sage_noalloc_device_status")
+    return int(code.value)
 
 
 def quantize(p: Params, device) -> None:
-    _check(lib().sage_quantize(ctypes.byref(p), _stream(device)), "sage_quantize")
+    _call("sage_quantize", p, device)
 
 
 def attn_quantized(p: Params, device) -> None:
-    _check(lib().sage_attn_quantized(ctypes.byref(p), _stream(device)), "sage_attn_quantized")
+    _call("sage_attn_quantized", p, device)
 
 
 def attn_fwd(p: Params, device) -> None:
-    _check(lib().sage_attn_fwd(ctypes.byref(p), _stream(device)), "sage_attn_fwd")
+    _call("sage_attn_fwd", p, device)
 
 
 def attn_fwd_prepass(p: Params, device) -> None:
-    _check(lib().sage_attn_fwd_prepass(ctypes.byref(p), _stream(device)), "sage_attn_fwd_prepass")
+    _call("sage_attn_fwd_prepass", p, device)
 
 
 def attn_fwd_attention(p: Params, device) -> None:
-    _check(lib().sage_attn_fwd_attention(ctypes.byref(p), _stream(device)), "sage_attn_fwd_attention")
+    _call("sage_attn_fwd_attention", p, device)
 
 
 def workspace_views(p: Params, workspace: torch.Tensor) -> dict:
@@ -393,12 +412,12 @@ def workspace_views(p: Params, workspace: torch.Tensor) -> dict:
         return workspace[off: off + n * esize].view(dtype).view(*shape)
 
     B, Hq, Hkv, D = p.B, p.Hq, p.Hkv, p.D
-    nqb, nkb = w.Nq_pad // 128, w.Nkv_pad // 64
+    nqb, nkb = w.Nq_pad // 128, w.Nkv_pad // 32
     out = dict(
         q8=view(w.q8, B * Hq * w.Nq_pad * w.Dp, torch.int8, (B, Hq, w.Nq_pad, w.Dp)),
         k8=view(w.k8, B * Hkv * w.Nkv_pad * w.Dp, torch.int8, (B, Hkv, w.Nkv_pad, w.Dp)),
         v8t=view(w.v8t, B * Hkv * D * w.Nkv_pad, torch.uint8, (B, Hkv, D, w.Nkv_pad)),
-        q_scale=view(w.q_scale, B * Hq * nqb, torch.float32, (B, Hq, nqb)),
+        q_scale=view(w.q_scale, B * Hq * w.Nq_pad, torch.float32, (B, Hq, w.Nq_pad)),
         k_scale=view(w.k_scale, B * Hkv * nkb, torch.float32, (B, Hkv, nkb)),
         v_scale=view(w.v_scale, B * Hkv * D, torch.float32, (B, Hkv, D)),
         mean_k=view(w.mean_k, B * Hkv * D, torch.float32, (B, Hkv, D)),
@@ -413,9 +432,15 @@ def workspace_views(p: Params, workspace: torch.Tensor) -> dict:
 
 
 def debug_dump_s(p: Params, b: int, h: int, qtile: int, ktile: int, device) -> torch.Tensor:
-    s = torch.empty((128, 128), dtype=torch.int32, device=device)
-    _check(lib().sage_debug_dump_s(ctypes.byref(p), b, h, qtile, ktile, ctypes.c_void_p(s.data_ptr()),
-                                   _stream(device)), "sage_debug_dump_s")
+    """The attention half of the pass in the S-dump build of the attention
+    kernel: returns the int32 S tile (qtile, ktile) of (b, h) as its softmax
+    warps read it (filled with -1 where the kernel computed no such tile);
+    writes p.out too."""
+    s = torch.full((128, 128), -1, dtype=torch.int32, device=device)
+    with torch.cuda.device(device):
+        _check(lib().sage_debug_dump_s(ctypes.byref(p), b, h, qtile, ktile,
+                                       ctypes.c_void_p(s.data_ptr()), _stream(device)),
+               "sage_debug_dump_s")
     return s
 
 
@@ -435,11 +460,21 @@ def debug_e4m3(x: torch.Tensor) -> torch.Tensor:
     return out
 
 
-def debug_mma_loop(ctas: int, iters: int, sink: torch.Tensor) -> None:
-    """sink: int32 device tensor with at least ctas + 1 entries (the last one is a status word)."""
+def debug_mma_loop(ctas: int, iters: int, sink: torch.Tensor, kind: int = 0) -> None:
+    """Back-to-back 8-bit MMAs (kind 0 INT8, kind 1 FP8 e4m3); sink: int32
+    device tensor with at least ctas + 1 entries (the last one is a status word)."""
     assert sink.dtype == torch.int32 and sink.numel() >= ctas + 1
-    _check(lib().sage_debug_mma_loop(ctas, iters, ctypes.c_void_p(sink.data_ptr()),
+    _check(lib().sage_debug_mma_loop(ctas, iters, kind, ctypes.c_void_p(sink.data_ptr()),
                                      _stream(sink.device)), "sage_debug_mma_loop")
+
+
+def debug_ex2(x: torch.Tensor) -> torch.Tensor:
+    """The attention kernel's exp2 applied to a float32 device tensor."""
+    assert x.is_cuda and x.dtype == torch.float32 and x.is_contiguous()
+    out = torch.empty_like(x)
+    _check(lib().sage_debug_ex2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+                                x.numel(), _stream(x.device)), "sage_debug_ex2")
+    return out
 
 
 def debug_wait_timeout(status: torch.Tensor) -> None:

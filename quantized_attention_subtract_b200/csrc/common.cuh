@@ -9,20 +9,21 @@ namespace sage {
 
 // Quantisation granularity and tiling.  The SageAttention pages fix
 // "per-block" quantisation of Q and K without block sizes ("sageattention"
-// package page, "What it is"); the reading taken: 128-token Q blocks (one
-// tensor-core M tile), 64-token K blocks (two per 128-key tile).
-constexpr int kQBlk = 128;
-constexpr int kKBlk = 64;
+// package page, "What it is") and name finer, per-thread granularity for
+// SageAttention2 (closerAI ComfyUI blog, part 4; "SageAttention2: Technical
+// report", section 1).  The reading taken: one INT8 scale per query token
+// (one softmax thread owns one query row), one per block of 32 keys (one per
+// 32-key section of that thread's exponent loop); query tiles and KV tiles
+// of 128 (one tensor-core M tile / N tile); Q's smoothing mean per 128-token
+// query tile.
+constexpr int kQTile = 128;
+constexpr int kKBlk = 32;
 constexpr int kKVTile = 128;
 
-// Online softmax with a lazily raised reference max m: a row's m is raised
-// to the tile max only when that exceeds m by more than kLazyLog2 (one
-// binade); O and l are rescaled only then.  Every logit s of a tile that did
-// not raise m satisfies s <= m + 1, so P is quantised as
-// e4m3(224 * 2^(s - m)) <= e4m3(448), e4m3's largest finite value.
-// kLog2P8Scale = fp32(log2(224)).
-constexpr float kLazyLog2 = 1.0f;
-constexpr float kLog2P8Scale = 7.807354927062988281f;   // 0x40F9D5DA
+// Online softmax, the plain rule: a row's running max m is raised to every
+// tile's max, and P is quantised as e4m3(448 * 2^(s - m)) <= 448, e4m3's
+// largest finite value.  kLog2P8 = fp32(log2(448)).
+constexpr float kLog2P8 = 8.807354927062988281f;        // 0x410CEAED
 constexpr float kLog2e = 1.44269502162933349609375f;    // fp32(log2 e), 0x3FB8AA3B
 
 // Fixed-point means: sum of rint(x * 2^24) in int64.
@@ -40,7 +41,7 @@ struct Workspace {
   long long *k_sum, *v_sum;      // fixed-point channel sums [B*Hkv][D]
   unsigned *v_max, *v_min;       // order-preserving keys of V channel max/min
   int *status;
-  int Dp, Nq_pad, Nkv_pad, nqb, nkb;
+  int Dp, Nq_pad, Nkv_pad, nqb, nkb;  // nqb: 128-row query tiles; nkb: 32-key K blocks
 };
 
 // Shapes / flags / strides of one call, as the kernels see them.
@@ -68,8 +69,8 @@ struct Problem {
   // work units that exist -- 128-row query tiles, 64-token and 128-token key
   // chunks -- (B + 1 entries each, device), and their grand totals, so that
   // kernels enumerate only units inside a sequence.
-  const int *pc_q128, *pc_kv64, *pc_kv128;
-  int tot_q128, tot_kv64, tot_kv128;
+  const int *pc_q128, *pc_kv64, *pc_kv128, *pc_q256;
+  int tot_q128, tot_kv64, tot_kv128, tot_q256;
   // Pre-pass loads of inputs whose tokens are strided (NHD, packed
   // variable-length batches, padded rows): 1 when the pre-pass reads that
   // tensor through the tensor maps of InputMaps (one box per unit) instead of
@@ -78,6 +79,11 @@ struct Problem {
   // a batch extent of 1.
   int k_map, v_map, q_map;
   int k_hn, v_hn, q_hn;
+  // Debug only (the S-dump instantiation of the attention kernel): the int32
+  // S tile of query tile dump_qt, KV tile dump_kt of (batch, head) dump_bh is
+  // copied row-major to s_dump[128 * 128] as the softmax warps read it.
+  int32_t *s_dump;
+  int dump_bh, dump_qt, dump_kt;
 };
 
 // Tensor maps of the caller's 16-bit inputs for the pre-pass: boxes of D
@@ -150,14 +156,14 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMa
                            cudaStream_t stream);
 cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
                              const CUtensorMap &tm_k, const CUtensorMap &tm_v, cudaStream_t stream);
-cudaError_t launch_dump_s(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
-                          const CUtensorMap &tm_k, int b, int h, int qtile, int ktile,
-                          int32_t *s_out, cudaStream_t stream);
+cudaError_t launch_attention_dump(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,
+                                  const CUtensorMap &tm_k, const CUtensorMap &tm_v, cudaStream_t stream);
 cudaError_t launch_debug_pv(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_v,
                             int b, int hkv, int ktile, const uint8_t *p8, float *o_out,
                             cudaStream_t stream);
 cudaError_t launch_debug_e4m3(const float *in, uint8_t *out, int64_t n, cudaStream_t stream);
-cudaError_t launch_mma_loop(int ctas, int iters, int32_t *sink, cudaStream_t stream);
+cudaError_t launch_mma_loop(int ctas, int iters, int kind, int32_t *sink, cudaStream_t stream);
+cudaError_t launch_debug_ex2(const float *in, float *out, int64_t n, cudaStream_t stream);
 cudaError_t launch_wait_timeout(int *status, cudaStream_t stream);
 
 }  // namespace sage

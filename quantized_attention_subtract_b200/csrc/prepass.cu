@@ -364,66 +364,64 @@ __global__ void kv_finalize_kernel(Problem pb, Workspace ws) {
   ws.v_inv[ci] = inv;
 }
 
-// Block-wide max of two non-negative values with one barrier: warp maxima go
-// into slot[0..1] by integer atomicMax (non-negative floats order like their
-// bits).  The slots must hold 0 before the call and stay untouched until
-// every thread has read them.
-__device__ __forceinline__ void block_max2_atomic(float &a, float &b, unsigned *slot) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
-  }
-  if ((threadIdx.x & 31) == 0) {
-    atomicMax(slot, __float_as_uint(a));
-    atomicMax(slot + 1, __float_as_uint(b));
-  }
-  __syncthreads();
-  a = __uint_as_float(slot[0]);
-  b = __uint_as_float(slot[1]);
-}
+// Lanes per row group of quantize_kernel: a power of two >= D / 8 (16-byte
+// chunks per row), so that a row group's lanes sit inside one warp and its
+// reductions are warp shuffles.  With D = 96 four lanes of each group idle.
+__host__ __device__ constexpr int quant_lanes(int D) { return D == 64 ? 8 : 16; }
 
 // INT8 codes of a thread's four rows (4 rg .. +3) x eight channels (8 c8 ..
-// +7) straight to a [128][Dp] tile in global memory; the 16 (D/8) threads of
-// a row write its D bytes contiguously, and threads c8 < (Dp - D) / 8 also
-// write the row's zero padding.
-__device__ __forceinline__ void store_codes(uint8_t *dst, int Dp, int D, int c8, int rg,
-                                            const float (&x)[4][8], float inv) {
+// +7), row r with reciprocal scale inv[r], straight to a [128][Dp] tile in
+// global memory: the lanes of a row write its Dp bytes contiguously, lanes
+// past the input's D / 8 chunks (not `live`) write the zero padding.
+__device__ __forceinline__ void store_codes(uint8_t *dst, int Dp, int c8, int rg, bool live,
+                                            const float (&x)[4][8], const float (&inv)[4]) {
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const uint32_t w0 = pack4_lo(int8_bits(x[r][0], inv), int8_bits(x[r][1], inv),
-                                 int8_bits(x[r][2], inv), int8_bits(x[r][3], inv));
-    const uint32_t w1 = pack4_lo(int8_bits(x[r][4], inv), int8_bits(x[r][5], inv),
-                                 int8_bits(x[r][6], inv), int8_bits(x[r][7], inv));
-    uint8_t *row = dst + (4 * rg + r) * Dp;
-    *reinterpret_cast<uint2 *>(row + 8 * c8) = make_uint2(w0, w1);
-    if (8 * c8 < Dp - D) *reinterpret_cast<uint2 *>(row + D + 8 * c8) = make_uint2(0u, 0u);
+    uint32_t w0 = 0u, w1 = 0u;
+    if (live) {
+      w0 = pack4_lo(int8_bits(x[r][0], inv[r]), int8_bits(x[r][1], inv[r]),
+                    int8_bits(x[r][2], inv[r]), int8_bits(x[r][3], inv[r]));
+      w1 = pack4_lo(int8_bits(x[r][4], inv[r]), int8_bits(x[r][5], inv[r]),
+                    int8_bits(x[r][6], inv[r]), int8_bits(x[r][7], inv[r]));
+    }
+    if (8 * c8 < Dp) *reinterpret_cast<uint2 *>(dst + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
   }
 }
 
-// Copy a finished [rows][row_bytes] tile from shared memory to a contiguous
-// global destination with 16-byte stores.
-__device__ __forceinline__ void store_tile(uint8_t *dst, const uint8_t *src, int bytes) {
-  for (int o = 16 * threadIdx.x; o < bytes; o += 16 * blockDim.x)
-    *reinterpret_cast<uint4 *>(dst + o) = *reinterpret_cast<const uint4 *>(src + o);
+// INT8 scale and reciprocal of a block with absolute maximum a (IEEE fp32
+// divisions): scale = a / 127, inv = 127 / a; both 0 below kTinyAmax.
+__device__ __forceinline__ void int8_scale(float a, float &scale, float &inv) {
+  scale = 0.f;
+  inv = 0.f;
+  if (a >= kTinyAmax) {
+    scale = __fdiv_rn(a, 127.0f);
+    inv = __fdiv_rn(127.0f, a);
+  }
 }
 
 // ------------------------------------------------------------ quantize
-// Persistent, grid <= 2 per SM, block 32 * (D / 8): thread t owns channels
-// 8 * (t % (D/8)) .. +7 of the four consecutive rows 4 * (t / (D/8)) .. +3 of
-// a 128-token tile.  Units: K and V tiles first, heads in reverse order
-// (those kv_stats read last may still be in L2), then Q blocks; block i takes
-// units i, i + grid, ...  Two input stages of 128 rows are kept in flight.
+// Persistent, grid <= 2 per SM, block 32 * L threads (L = quant_lanes(D)):
+// thread t owns channels 8 * (t % L) .. +7 of the four consecutive rows
+// 4 * (t / L) .. +3 of a 128-token tile.  Units: K and V tiles first, heads
+// in reverse order (those kv_stats read last may still be in L2), then Q
+// tiles; block i takes units i, i + grid, ...  Two input stages of 128 rows
+// are kept in flight.
+//   K tile: K' = K - mean_k; four INT8 blocks of 32 rows (8 row groups, a
+//           whole number of warps each): block amax by warp shuffles and one
+//           shared atomic per warp, one barrier.
+//   Q tile: optional smoothing by the tile's channel mean; one INT8 scale per
+//           row: row amax by shuffles among the row group's lanes, no barrier.
+//   V tile: V' = V - mean_v, FP8 per channel, transposed through shared memory.
 constexpr int kQuantStages = 2;
 
 struct QUnit {
-  int kind;  // 0 = K tile, 1 = V tile, 2 = Q block
+  int kind;  // 0 = K tile, 1 = V tile, 2 = Q tile
   int bh, t, b, h, r0, nvalid;
   const uint16_t *src;
   long long stride;
 };
 
-// Units of quantize_kernel: K and V tiles (both), then Q blocks unless the
+// Units of quantize_kernel: K and V tiles (both), then Q tiles unless the
 // attention kernel quantises Q; variable-length batches count only the tiles
 // inside a sequence.
 __host__ __device__ __forceinline__ long long quant_units(const Problem &pb, const Workspace &ws) {
@@ -485,8 +483,8 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
     }
     q.b = q.bh / pb.Hq;
     q.h = q.bh % pb.Hq;
-    q.r0 = q.t * kQBlk;
-    q.nvalid = max(0, min(kQBlk, nq_of(pb, q.b) - q.r0));
+    q.r0 = q.t * kQTile;
+    q.nvalid = max(0, min(kQTile, nq_of(pb, q.b) - q.r0));
     q.src = pb.q + q_off(pb, q.b) + q.h * pb.qs_h + q.r0 * pb.qs_n;
     q.stride = pb.qs_n;
   }
@@ -502,23 +500,23 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
                                                           const __grid_constant__ CUtensorMap mq) {
   extern __shared__ __align__(1024) uint8_t sm_q[];
   if (smem_misaligned(sm_q, ws.status)) return;
-  const int D = pb.D, Dp = ws.Dp, C8 = D / 8, rowb = 2 * D;
-  const int c8 = threadIdx.x % C8, rg = threadIdx.x / C8;  // rows 4 rg .. 4 rg + 3
+  const int D = pb.D, Dp = ws.Dp, C8 = D / 8, L = quant_lanes(D), rowb = 2 * D;
+  const int c8 = threadIdx.x % L, rg = threadIdx.x / L;  // rows 4 rg .. 4 rg + 3
+  const bool live = c8 < C8;                              // lane holds input channels
   const int stage_bytes = 128 * rowb;
   uint8_t *tile = sm_q + kQuantStages * stage_bytes;        // output codes [128][128]
   uint64_t *bars = reinterpret_cast<uint64_t *>(tile + 128 * 128);
   unsigned long long *colsum = reinterpret_cast<unsigned long long *>(bars + 4);
   float *chan = reinterpret_cast<float *>(colsum + 128);
-  float *scratch = chan + 128;                               // 66 floats
-  unsigned *mslot = reinterpret_cast<unsigned *>(scratch + 66);  // [2 parities][2]
-  QUnit *desc = reinterpret_cast<QUnit *>(scratch + 72);    // [stages + 1]
+  unsigned *mslot = reinterpret_cast<unsigned *>(chan + 128);  // [2 parities][4 K blocks]
+  QUnit *desc = reinterpret_cast<QUnit *>(mslot + 8);        // [stages + 1]
   const uint32_t s_base = smem_u32(sm_q), b_base = smem_u32(bars);
-  // K and V tiles, then Q blocks (skipped when the attention kernel quantises Q)
+  // K and V tiles, then Q tiles (skipped when the attention kernel quantises Q)
   const long long nunits = quant_units(pb, ws);
   if (threadIdx.x == 0) {
     for (int i = 0; i < kQuantStages; ++i) mbar_init(b_base + 8 * i, 1);
     fence_mbar_init();
-    for (int i = 0; i < 4; ++i) mslot[i] = 0u;
+    for (int i = 0; i < 8; ++i) mslot[i] = 0u;
   }
   __syncthreads();
   // Unit descriptors are decoded once, by thread 0, into a ring of
@@ -559,18 +557,15 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
     const int st = it % kQuantStages;
     if (!block_wait(b_base + 8 * st, (it / kQuantStages) & 1, ws.status)) { ok = false; break; }
     const QUnit q = desc[it % kSlots];
-    // block-max slots: this unit uses parity it & 1; the other parity (last
+    // K-block max slots: this unit uses parity it & 1; the other parity (last
     // read in iteration it - 1) is cleared for the next unit
-    unsigned *mx = mslot + 2 * (it & 1);
-    if (threadIdx.x == 0) {
-      mslot[2 * ((it + 1) & 1)] = 0u;
-      mslot[2 * ((it + 1) & 1) + 1] = 0u;
-    }
+    unsigned *mx = mslot + 4 * (it & 1);
+    if (threadIdx.x < 4) mslot[4 * ((it + 1) & 1) + threadIdx.x] = 0u;
     const uint8_t *stage = sm_q + st * stage_bytes;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int row = 4 * rg + r;
-      if (row < q.nvalid) decode8(*reinterpret_cast<const uint4 *>(stage + row * rowb + 16 * c8), pb.bf16, x[r]);
+      if (live && row < q.nvalid) decode8(*reinterpret_cast<const uint4 *>(stage + row * rowb + 16 * c8), pb.bf16, x[r]);
       else
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[r][e] = 0.f;
@@ -582,49 +577,46 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
     if (un < nunits) issue(*dn, st);
 
     if (q.kind == 0) {
-      // ---------------- K tile: K' = K - mean_k, two INT8 blocks of 64
-      float mean[8];
-      {
-        const float4 *mk = reinterpret_cast<const float4 *>(ws.mean_k + (long long)q.bh * D + 8 * c8);
-        const float4 m0 = __ldg(mk), m1 = __ldg(mk + 1);
+      // ---------------- K tile: K' = K - mean_k, four INT8 blocks of 32 rows
+      float mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (live) {
+        const float4 *mk4 = reinterpret_cast<const float4 *>(ws.mean_k + (long long)q.bh * D + 8 * c8);
+        const float4 m0 = __ldg(mk4), m1 = __ldg(mk4 + 1);
         mean[0] = m0.x; mean[1] = m0.y; mean[2] = m0.z; mean[3] = m0.w;
         mean[4] = m1.x; mean[5] = m1.y; mean[6] = m1.z; mean[7] = m1.w;
       }
       float a = 0.f;
 #pragma unroll
       for (int r = 0; r < 4; ++r)
-        if (4 * rg + r < q.nvalid)
+        if (live && 4 * rg + r < q.nvalid)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             x[r][e] = __fsub_rn(x[r][e], mean[e]);
             a = fmaxf(a, fabsf(x[r][e]));
           }
-      // rows 0..63 belong to block 2 t, rows 64..127 to 2 t + 1
-      float a0 = rg < 16 ? a : 0.f, a1 = rg < 16 ? 0.f : a;
-      block_max2_atomic(a0, a1, mx);
-      float inv0 = 0.f, inv1 = 0.f, s0 = 0.f, s1 = 0.f;
-      if (a0 >= kTinyAmax) {
-        s0 = __fdiv_rn(a0, 127.0f);
-        inv0 = __fdiv_rn(127.0f, a0);
+      // rows 32 k .. 32 k + 31 (row groups 8 k .. 8 k + 7) form block k; each
+      // warp lies inside one block.  Non-negative floats order like their bits.
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if ((threadIdx.x & 31) == 0) atomicMax(mx + rg / 8, __float_as_uint(a));
+      __syncthreads();
+      float inv[4], sc;
+      int8_scale(__uint_as_float(mx[rg / 8]), sc, inv[0]);
+      inv[1] = inv[2] = inv[3] = inv[0];
+      if (threadIdx.x < 4) {
+        float s4, i4;
+        int8_scale(__uint_as_float(mx[threadIdx.x]), s4, i4);
+        ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 4 * q.t + threadIdx.x] = s4;
       }
-      if (a1 >= kTinyAmax) {
-        s1 = __fdiv_rn(a1, 127.0f);
-        inv1 = __fdiv_rn(127.0f, a1);
-      }
-      if (threadIdx.x == 0) {
-        ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 2 * q.t] = s0;
-        ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 2 * q.t + 1] = s1;
-      }
-      const float inv = rg < 16 ? inv0 : inv1;
-      store_codes(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, Dp, D,
-                  c8, rg, x, inv);
+      store_codes(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, Dp,
+                  c8, rg, live, x, inv);
     } else if (q.kind == 1) {
       // ---------------- V tile: V' = V - mean_v, FP8 per channel, transposed
-      float mean[8], inv[8];
-      {
-        const float4 *mv = reinterpret_cast<const float4 *>(ws.mean_v + (long long)q.bh * D + 8 * c8);
-        const float4 *iv = reinterpret_cast<const float4 *>(ws.v_inv + (long long)q.bh * D + 8 * c8);
-        const float4 m0 = __ldg(mv), m1 = __ldg(mv + 1), i0 = __ldg(iv), i1 = __ldg(iv + 1);
+      float mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, inv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (live) {
+        const float4 *mv4 = reinterpret_cast<const float4 *>(ws.mean_v + (long long)q.bh * D + 8 * c8);
+        const float4 *iv4 = reinterpret_cast<const float4 *>(ws.v_inv + (long long)q.bh * D + 8 * c8);
+        const float4 m0 = __ldg(mv4), m1 = __ldg(mv4 + 1), i0 = __ldg(iv4), i1 = __ldg(iv4 + 1);
         mean[0] = m0.x; mean[1] = m0.y; mean[2] = m0.z; mean[3] = m0.w;
         mean[4] = m1.x; mean[5] = m1.y; mean[6] = m1.z; mean[7] = m1.w;
         inv[0] = i0.x; inv[1] = i0.y; inv[2] = i0.z; inv[3] = i0.w;
@@ -640,20 +632,22 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       // Transposed tile [D][128 keys] as 32 words per channel row; the word of
       // keys 4 rg .. 4 rg + 3 of channel c sits at position (rg + rot * c8) % 32,
       // which puts the 32 lanes of a warp on 32 different banks.
-      const int rot = 32 / (C8 == 12 ? 16 : C8);
+      const int rot = 32 / L;
       uint32_t *tw = reinterpret_cast<uint32_t *>(tile);
+      if (live) {
 #pragma unroll
-      for (int e = 0; e < 8; e += 2) {
-        uint32_t w_lo = 0, w_hi = 0;
+        for (int e = 0; e < 8; e += 2) {
+          uint32_t w_lo = 0, w_hi = 0;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const uint32_t pr = e4m3x2(x[r][e], x[r][e + 1]);
-          w_lo |= (pr & 0xFFu) << (8 * r);
-          w_hi |= (pr >> 8) << (8 * r);
+          for (int r = 0; r < 4; ++r) {
+            const uint32_t pr = e4m3x2(x[r][e], x[r][e + 1]);
+            w_lo |= (pr & 0xFFu) << (8 * r);
+            w_hi |= (pr >> 8) << (8 * r);
+          }
+          const int pos = (rg + rot * c8) & 31;
+          tw[(8 * c8 + e) * 32 + pos] = w_lo;
+          tw[(8 * c8 + e + 1) * 32 + pos] = w_hi;
         }
-        const int pos = (rg + rot * c8) & 31;
-        tw[(8 * c8 + e) * 32 + pos] = w_lo;
-        tw[(8 * c8 + e + 1) * 32 + pos] = w_hi;
       }
       __syncthreads();
       uint8_t *dst = ws.v8t + (long long)q.bh * D * ws.Nkv_pad + q.r0;
@@ -668,17 +662,19 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
         *reinterpret_cast<uint4 *>(dst + (long long)c * ws.Nkv_pad + 16 * qq) = o;
       }
     } else {
-      // ---------------- Q block: optional block mean, INT8 per block
+      // ---------------- Q tile: optional smoothing mean, one INT8 scale per row
       if (pb.smooth_q) {
         if (int(threadIdx.x) < D) colsum[threadIdx.x] = 0ull;
         __syncthreads();
+        if (live) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          long long s = 0;
+          for (int e = 0; e < 8; ++e) {
+            long long s = 0;
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-            if (4 * rg + r < q.nvalid) s += fixed_point(x[r][e]);
-          atomicAdd(&colsum[8 * c8 + e], (unsigned long long)s);
+            for (int r = 0; r < 4; ++r)
+              if (4 * rg + r < q.nvalid) s += fixed_point(x[r][e]);
+            atomicAdd(&colsum[8 * c8 + e], (unsigned long long)s);
+          }
         }
         __syncthreads();
         if (int(threadIdx.x) < D) {
@@ -687,26 +683,35 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
           ws.mq[((long long)q.bh * ws.nqb + q.t) * D + threadIdx.x] = m;
         }
         __syncthreads();
+        if (live) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-          if (4 * rg + r < q.nvalid)
+          for (int r = 0; r < 4; ++r)
+            if (4 * rg + r < q.nvalid)
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], chan[8 * c8 + e]);
+              for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], chan[8 * c8 + e]);
+        }
       }
-      float a = 0.f, unused = 0.f;
+      float a[4], inv[4], sc[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r)
+      for (int r = 0; r < 4; ++r) {
+        a[r] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(x[r][e]));
-      block_max2_atomic(a, unused, mx);
-      float inv = 0.f, scale = 0.f;
-      if (a >= kTinyAmax) {
-        scale = __fdiv_rn(a, 127.0f);
-        inv = __fdiv_rn(127.0f, a);
+        for (int e = 0; e < 8; ++e) a[r] = fmaxf(a[r], fabsf(x[r][e]));
       }
-      if (threadIdx.x == 0) ws.q_scale[(long long)q.bh * ws.nqb + q.t] = scale;
-      store_codes(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, Dp, D,
-                  c8, rg, x, inv);
+      // row amax over the row group's L lanes (aligned inside the warp)
+#pragma unroll
+      for (int o = L / 2; o > 0; o >>= 1)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) a[r] = fmaxf(a[r], __shfl_xor_sync(0xffffffffu, a[r], o));
+#pragma unroll
+      for (int r = 0; r < 4; ++r) int8_scale(a[r], sc[r], inv[r]);
+      if (c8 < 4) {
+        // lane c8 of the group stores row 4 rg + c8's scale (0 past nvalid)
+        const float s = c8 == 0 ? sc[0] : c8 == 1 ? sc[1] : c8 == 2 ? sc[2] : sc[3];
+        ws.q_scale[(long long)q.bh * ws.Nq_pad + q.r0 + 4 * rg + c8] = s;
+      }
+      store_codes(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, Dp,
+                  c8, rg, live, x, inv);
     }
     // The V transpose tile is rewritten only after the next unit's first
     // barrier, which every thread reaches after its reads of this one.
@@ -795,8 +800,8 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMa
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // quantize: persistent, 2 blocks per SM
-  // stages | output tile | 4 barriers | colsum[128] | chan[128] | scratch[72] | desc[stages + 1]
-  const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 72 * 4 +
+  // stages | output tile | 4 barriers | colsum[128] | chan[128] | K-block max slots[8] | desc[stages + 1]
+  const size_t q_smem = kQuantStages * 128 * rowb + 128 * 128 + 32 + 128 * 8 + 128 * 4 + 8 * 4 +
                         (kQuantStages + 1) * sizeof(QUnit);
   const bool maps = pb.k_map || pb.v_map || pb.q_map;
   auto qk = pb.cu_q ? (maps ? quantize_kernel<true, true> : quantize_kernel<true, false>)
@@ -806,7 +811,7 @@ cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMa
   const long long nblk = quant_units(pb, ws);
   const unsigned g2 = (unsigned)std::min<long long>(nblk, 2LL * sms);
   if (g2 > 0) {
-    qk<<<g2, 32 * (pb.D / 8), q_smem, stream>>>(pb, ws, im.k128, im.v128, im.q128);
+    qk<<<g2, 32 * quant_lanes(pb.D), q_smem, stream>>>(pb, ws, im.k128, im.v128, im.q128);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

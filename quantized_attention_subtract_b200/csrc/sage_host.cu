@@ -44,7 +44,7 @@ sage_status_t check_shape(const sage_attn_params_t *p) {
   if (p->Hq % p->Hkv != 0) return SAGE_ERR_INVALID_ARG;
   if (p->Nq > 0 && p->Nkv < 1) return SAGE_ERR_INVALID_ARG;
   if (!is_flag(p->is_causal) || !is_flag(p->smooth_k) || !is_flag(p->smooth_q) ||
-      !is_flag(p->smooth_v) || !is_flag(p->fuse_q))
+      !is_flag(p->smooth_v))
     return SAGE_ERR_INVALID_ARG;
   if (!(p->sm_scale == p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
   // TMA row coordinates and kernel indices are 32-bit
@@ -79,7 +79,7 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.Nq_pad = int((p->Nq + 127) / 128 * 128);
   L.Nkv_pad = int((p->Nkv + 127) / 128 * 128);
   L.nqb = L.Nq_pad / 128;
-  L.nkb = L.Nkv_pad / 64;
+  L.nkb = L.Nkv_pad / kKBlk;
   const size_t BHq = size_t(p->B) * p->Hq, BHk = size_t(p->B) * p->Hkv, D = size_t(p->D);
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -90,8 +90,8 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.off_q8 = take(BHq * L.Nq_pad * L.Dp);
   L.off_k8 = take(BHk * L.Nkv_pad * L.Dp);
   L.off_v8t = take(BHk * D * L.Nkv_pad);
-  L.off_qs = take(BHq * L.nqb * sizeof(float));
-  L.off_ks = take(BHk * L.nkb * sizeof(float));
+  L.off_qs = take(BHq * L.Nq_pad * sizeof(float));   // one scale per query token
+  L.off_ks = take(BHk * L.nkb * sizeof(float));      // one per 32 keys
   L.off_vs = take(BHk * D * sizeof(float));
   L.off_mk = take(BHk * D * sizeof(float));
   L.off_mv = take(BHk * D * sizeof(float));
@@ -105,8 +105,8 @@ Layout make_layout(const sage_attn_params_t *p) {
   L.off_vmin = take(BHk * D * sizeof(unsigned));
   L.off_vinv = take(BHk * D * sizeof(float));
   L.off_status = take(16);
-  // offsets and running unit totals of a variable-length batch: 5 x (B + 1)
-  L.off_cu = is_varlen(p) ? take(5 * (size_t(p->B) + 1) * sizeof(int32_t)) : 0;
+  // offsets and running unit totals of a variable-length batch: 6 x (B + 1)
+  L.off_cu = is_varlen(p) ? take(6 * (size_t(p->B) + 1) * sizeof(int32_t)) : 0;
   if (p->smooth_q) {
     L.off_mq = take(BHq * L.nqb * D * sizeof(float));
     L.off_dsk = take(BHq * L.nqb * size_t(L.Nkv_pad) * sizeof(float));
@@ -257,29 +257,6 @@ struct Maps {
   CUtensorMap q, k, v;
 };
 
-// Tensor map of the caller's 16-bit Q for the attention kernel's fused
-// quantisation: dimensions (D, Nq, Hq, B), or (D, Hq, Nq, B) when the head
-// stride is the smaller one, so the strides increase; box 32 channels x 128
-// tokens (x 1 x 1), 64-byte swizzle, zero fill past Nq.  Returns false when
-// the driver rejects the strides (the caller then quantises Q in the
-// pre-pass instead).
-bool make_q_input_map(const Problem &pb, CUtensorMap *m, int *hn) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const bool head_inner = pb.qs_h < pb.qs_n;
-  *hn = head_inner ? 1 : 0;
-  const cuuint64_t dims[4] = {cuuint64_t(pb.D), cuuint64_t(head_inner ? pb.Hq : pb.Nq),
-                              cuuint64_t(head_inner ? pb.Nq : pb.Hq), cuuint64_t(pb.B)};
-  const cuuint64_t strides[3] = {cuuint64_t(2 * (head_inner ? pb.qs_h : pb.qs_n)),
-                                 cuuint64_t(2 * (head_inner ? pb.qs_n : pb.qs_h)), cuuint64_t(2 * pb.qs_b)};
-  const cuuint32_t box[4] = {32, head_inner ? 1u : 128u, head_inner ? 128u : 1u, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return fn(m, pb.bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
-            const_cast<uint16_t *>(pb.q), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Tensor map of a caller's 16-bit input (element strides s_b, s_h, s_n; the
 // channel stride is 1) for the pre-pass: dimensions (D, N, H, B), or
 // (D, H, N, B) when the head stride is the smaller one, so the strides
@@ -331,7 +308,7 @@ void make_input_maps(Problem &pb, InputMaps &im, long long nq_tot, long long nkv
     pb.v_map = 1;
     pb.v_hn = hn0;
   }
-  if (pb.qs_n != pb.D && !pb.q_fused &&
+  if (pb.qs_n != pb.D &&
       make_input_map(pb.q, pb.bf16, pb.D, pb.qs_b, pb.qs_h, pb.qs_n, pb.Hq, Nq, Bm, 128, &im.q128, &hn0)) {
     pb.q_map = 1;
     pb.q_hn = hn0;
@@ -361,13 +338,8 @@ sage_status_t validate(const sage_attn_params_t *p, bool need_inputs, bool need_
   return check_device();
 }
 
-// pre / attn: which half of the pass to enqueue.  whole_pass: the halves of
-// sage_attn_fwd, where Q is quantised inside the attention kernel when the
-// caller asks for it (fuse_q), Q is not smoothed and the driver accepts a
-// tensor map of the caller's Q; the separate pre-pass and attention calls
-// always go through the workspace.
-sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, bool attn,
-                  bool whole_pass) {
+// pre / attn: which half of the pass to enqueue (both for sage_attn_fwd).
+sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, bool attn) {
   // No queries: nothing to compute and no pointer is read (empty tensors
   // may have null data pointers).
   sage_status_t s = check_shape(p);
@@ -382,12 +354,13 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
   long long nq_tot = 0, nkv_tot = 0;  // packed token counts (variable-length batches)
   if (is_varlen(p)) {
     // The kernels read the (validated) sequence offsets from the workspace,
-    // with the running totals of each sequence's query tiles (128 rows) and
-    // key chunks (64 and 128 tokens), so that they enumerate only units
-    // inside a sequence.
+    // with the running totals of each sequence's query tiles (128 rows),
+    // query-tile pairs (256 rows) and key chunks (64 and 128 tokens), so that
+    // they enumerate only units inside a sequence.
     const int B = p->B;
-    std::vector<int32_t> h(5 * size_t(B + 1), 0);
-    int32_t *cq = h.data(), *ck = cq + B + 1, *pq = ck + B + 1, *p64 = pq + B + 1, *p128 = p64 + B + 1;
+    std::vector<int32_t> h(6 * size_t(B + 1), 0);
+    int32_t *cq = h.data(), *ck = cq + B + 1, *pq = ck + B + 1, *p64 = pq + B + 1, *p128 = p64 + B + 1,
+            *p256 = p128 + B + 1;
     for (int b = 0; b <= B; ++b) {
       cq[b] = p->cu_seqlens_q[b];
       ck[b] = p->cu_seqlens_kv[b];
@@ -397,6 +370,7 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
       pq[b + 1] = pq[b] + (lq + 127) / 128;
       p64[b + 1] = p64[b] + (lk + 63) / 64;
       p128[b + 1] = p128[b] + (lk + 127) / 128;
+      p256[b + 1] = p256[b] + ((lq + 127) / 128 + 1) / 2;  // pairs of query tiles
     }
     int32_t *d = reinterpret_cast<int32_t *>(static_cast<uint8_t *>(p->workspace) + L.off_cu);
     // pageable source: the copy has read h before the call returns
@@ -407,23 +381,15 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
     pb.pc_q128 = d + 2 * (B + 1);
     pb.pc_kv64 = d + 3 * (B + 1);
     pb.pc_kv128 = d + 4 * (B + 1);
+    pb.pc_q256 = d + 5 * (B + 1);
+    pb.tot_q256 = p256[B];
     pb.tot_q128 = pq[B];
     pb.tot_kv64 = p64[B];
     pb.tot_kv128 = p128[B];
     nq_tot = cq[B];
     nkv_tot = ck[B];
   }
-  // With fuse_q the whole pass quantises Q inside the attention kernel (it
-  // still writes q8 and q_scale to the workspace) and the pre-pass skips Q.
-  // The decision depends only on p, so both halves agree.
   Maps m;
-  if (whole_pass && p->fuse_q && !p->smooth_q && !is_varlen(p)) {
-    int hn = 0;
-    if (make_q_input_map(pb, &m.q, &hn)) {
-      pb.q_fused = 1;
-      pb.q_map_hn = hn;
-    }
-  }
   if (pre && cudaMemsetAsync(ws.status, 0, sizeof(int), st) != cudaSuccess) return SAGE_ERR_CUDA;
   if (pre) {
     InputMaps im;
@@ -432,9 +398,7 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
     if (launch_prepass(pb, ws, im, st) != cudaSuccess) return SAGE_ERR_CUDA;
   }
   if (attn) {
-    CUtensorMap q_input = m.q;
     if (!make_maps(p, ws, m)) return SAGE_ERR_CUDA;
-    if (pb.q_fused) m.q = q_input;
     if (launch_attention(pb, ws, m.q, m.k, m.v, st) != cudaSuccess) return SAGE_ERR_CUDA;
   }
   return SAGE_OK;
@@ -444,24 +408,67 @@ sage_status_t run(const sage_attn_params_t *p, sage_stream_t stream, bool pre, b
 // array per device that loads the library, alive until the process exits.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[SAGE_NOALLOC_MAX_WORKSPACE_BYTES];
 
-// Device address of g_noalloc_scratch per device ordinal, looked up once with
-// that device current.  In host code the array's name is only a host-side
-// stand-in, never a device address.
+// Device address of g_noalloc_scratch, looked up with the device current and
+// cached per device ordinal together with the context it was looked up in:
+// after a device reset the module is loaded again (possibly elsewhere) in a
+// new primary context, so a changed context triggers a fresh lookup.  In host
+// code the array's name is only a host-side stand-in, never a device address.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 void *g_noalloc_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 
 sage_status_t noalloc_scratch(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
+  // a first lookup lets the runtime create or bind the device's primary
+  // context; the context is read after it
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void *ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SAGE_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (g_noalloc_ptr[dev]) {
+    if (!get || get(&ctx) != CUDA_SUCCESS) return SAGE_ERR_CUDA;
+    if (ctx == g_noalloc_ctx[dev]) {
+      *out = g_noalloc_ptr[dev];
+      return SAGE_OK;
+    }
   }
-  *out = g_noalloc_ptr[dev];
+  void *ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return SAGE_ERR_CUDA;
+  if (!get || get(&ctx) != CUDA_SUCCESS || !ctx) return SAGE_ERR_CUDA;
+  g_noalloc_ptr[dev] = ptr;
+  g_noalloc_ctx[dev] = ctx;
+  *out = ptr;
+  return SAGE_OK;
+}
+
+// The params of a call redirected to the library scratch.
+sage_status_t noalloc_params(const sage_attn_params_t *p, sage_attn_params_t *q) {
+  sage_status_t s = check_shape(p);
+  if (s != SAGE_OK) return s;
+  if (make_layout(p).total > SAGE_NOALLOC_MAX_WORKSPACE_BYTES) return SAGE_ERR_WORKSPACE;
+  if ((s = check_device()) != SAGE_OK) return s;
+  void *scratch = nullptr;
+  if ((s = noalloc_scratch(&scratch)) != SAGE_OK) return s;
+  *q = *p;
+  q->workspace = scratch;
+  q->workspace_bytes = SAGE_NOALLOC_MAX_WORKSPACE_BYTES;
   return SAGE_OK;
 }
 
@@ -517,51 +524,59 @@ sage_status_t sage_workspace_view(const sage_attn_params_t *p, sage_workspace_vi
 }
 
 sage_status_t sage_attn_fwd(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, true, true, true);
+  return run(p, stream, true, true);
 }
 
 sage_status_t sage_attn_fwd_prepass(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, true, false, true);
+  return run(p, stream, true, false);
 }
 
 sage_status_t sage_attn_fwd_attention(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, false, true, true);
+  return run(p, stream, false, true);
 }
 
 sage_status_t sage_attn_fwd_noalloc(const sage_attn_params_t *p, sage_stream_t stream) {
-  sage_status_t s = check_shape(p);
+  sage_attn_params_t q;
+  const sage_status_t s = noalloc_params(p, &q);
   if (s != SAGE_OK) return s;
-  if (make_layout(p).total > SAGE_NOALLOC_MAX_WORKSPACE_BYTES) return SAGE_ERR_WORKSPACE;
-  if ((s = check_device()) != SAGE_OK) return s;
-  void *scratch = nullptr;
-  if ((s = noalloc_scratch(&scratch)) != SAGE_OK) return s;
-  sage_attn_params_t q = *p;
-  q.workspace = scratch;
-  q.workspace_bytes = SAGE_NOALLOC_MAX_WORKSPACE_BYTES;
-  return run(&q, stream, true, true, true);
+  return run(&q, stream, true, true);
+}
+
+sage_status_t sage_noalloc_device_status(const sage_attn_params_t *p, int32_t *code) {
+  if (!code) return SAGE_ERR_INVALID_ARG;
+  sage_attn_params_t q;
+  const sage_status_t s = noalloc_params(p, &q);
+  if (s != SAGE_OK) return s;
+  return sage_get_device_status(&q, code);
 }
 
 sage_status_t sage_quantize(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, true, false, false);
+  return run(p, stream, true, false);
 }
 
 sage_status_t sage_attn_quantized(const sage_attn_params_t *p, sage_stream_t stream) {
-  return run(p, stream, false, true, false);
+  return run(p, stream, false, true);
 }
 
 sage_status_t sage_debug_dump_s(const sage_attn_params_t *p, int32_t b, int32_t h, int32_t qtile,
                                 int32_t ktile, int32_t *s_out, sage_stream_t stream) {
-  Layout L;
-  sage_status_t s = validate(p, false, false, L);
+  sage_status_t s = check_shape(p);
   if (s != SAGE_OK) return s;
+  if (p->Nq == 0 || is_varlen(p)) return SAGE_ERR_INVALID_ARG;
+  Layout L;
+  if ((s = validate(p, false, true, L)) != SAGE_OK) return s;
   if (!s_out || b < 0 || b >= p->B || h < 0 || h >= p->Hq || qtile < 0 || qtile >= L.nqb ||
       ktile < 0 || ktile >= L.Nkv_pad / 128)
     return SAGE_ERR_INVALID_ARG;
   const Workspace ws = make_workspace(p, L);
   Maps m;
   if (!make_maps(p, ws, m)) return SAGE_ERR_CUDA;
-  return launch_dump_s(make_problem(p), ws, m.q, m.k, b, h, qtile, ktile, s_out,
-                       reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  Problem pb = make_problem(p);
+  pb.s_dump = s_out;
+  pb.dump_bh = b * p->Hq + h;
+  pb.dump_qt = qtile;
+  pb.dump_kt = ktile;
+  return launch_attention_dump(pb, ws, m.q, m.k, m.v, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SAGE_OK
              : SAGE_ERR_CUDA;
 }
@@ -592,12 +607,21 @@ sage_status_t sage_debug_e4m3(const float *in, uint8_t *out, int64_t n, sage_str
              : SAGE_ERR_CUDA;
 }
 
-sage_status_t sage_debug_mma_loop(int32_t ctas, int32_t iters, int32_t *sink,
+sage_status_t sage_debug_mma_loop(int32_t ctas, int32_t iters, int32_t kind, int32_t *sink,
                                   sage_stream_t stream) {
-  if (ctas < 1 || iters < 1 || !sink) return SAGE_ERR_INVALID_ARG;
+  if (ctas < 1 || iters < 1 || (kind != 0 && kind != 1) || !sink) return SAGE_ERR_INVALID_ARG;
   sage_status_t s = check_device();
   if (s != SAGE_OK) return s;
-  return launch_mma_loop(ctas, iters, sink, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_mma_loop(ctas, iters, kind, sink, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
+
+sage_status_t sage_debug_ex2(const float *in, float *out, int64_t n, sage_stream_t stream) {
+  if (n < 0 || (n > 0 && (!in || !out))) return SAGE_ERR_INVALID_ARG;
+  sage_status_t s = check_device();
+  if (s != SAGE_OK) return s;
+  return launch_debug_ex2(in, out, n, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SAGE_OK
              : SAGE_ERR_CUDA;
 }

@@ -9,12 +9,12 @@ import oracle
 from quantized_attention_subtract_b200 import binding
 from quantized_attention_subtract_b200.workloads import Workload, generate
 
-# Output tolerances of the GPU path against the oracle's mirror of the same
-# quantised algorithm, as the task states them: max |diff| <= 2e-2 and cosine
-# similarity >= 0.9999.  Against exact fp64 attention the quantisation itself
-# costs ~3.5-4.5% relative L1 on iid inputs (FP8 P and V each contribute
-# ~2.4%); the bound used is 0.06 relative L1 and cosine >= 0.998 on inputs
-# without channel outliers.
+# Output tolerances of the GPU path against the oracle (the plain online
+# softmax of the quantised method): max |diff| <= 2e-2 and cosine similarity
+# >= 0.9999.  Against exact fp64 attention the quantisation itself costs
+# ~3.7% relative L1 on iid inputs: FP8 P and FP8 V each contribute the e4m3
+# rms rounding error of ~2.65% (pinned in the oracle's CPU tests), INT8 Q K^T
+# ~1%; the bound used is 0.06 relative L1 and cosine >= 0.998.
 MIRROR_MAX_ABS = 2e-2
 MIRROR_COS = 0.9999
 EXACT_REL_L1 = 0.06
@@ -35,12 +35,12 @@ def to_device(bits: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
 class DeviceRun:
     """Inputs on the device, the output, the workspace and its views."""
 
-    def __init__(self, w: Workload, q, k, v, run_attention: bool = True, fuse_q: bool = False):
+    def __init__(self, w: Workload, q, k, v, run_attention: bool = True):
         self.w = w
         self.q, self.k, self.v = (to_device(x, w.dtype) for x in (q, k, v))
         self.out = torch.empty_like(self.q)
         self.p = binding.make_params(self.q, self.k, self.v, self.out, w.layout, w.is_causal, None,
-                                     w.smooth_k, w.smooth_q, w.smooth_v, fuse_q=fuse_q)
+                                     w.smooth_k, w.smooth_q, w.smooth_v)
         self.ws = binding.alloc_workspace(self.p, self.q.device)
         if run_attention:
             binding.attn_fwd(self.p, self.q.device)
@@ -54,11 +54,11 @@ class DeviceRun:
         return self.out.double().cpu().numpy()
 
 
-def run_both(w: Workload, seed=None, fuse_q: bool = False):
+def run_both(w: Workload, seed=None):
     q, k, v = generate(w, seed)
     pr = oracle_problem(w)
     pre = oracle.prepass(pr, q, k, v)
-    g = DeviceRun(w, q, k, v, fuse_q=fuse_q)
+    g = DeviceRun(w, q, k, v)
     return q, k, v, pr, pre, g
 
 
@@ -74,7 +74,8 @@ def assert_prepass_bit_exact(w: Workload, pre: dict, g: DeviceRun):
     v8 = V["v8t"].transpose(0, 1, 3, 2)
     assert np.array_equal(v8[:, :, :Nkv], pre["v8"]), "v8"
     assert not v8[:, :, Nkv:].any(), "v8 padding"
-    assert np.array_equal(V["q_scale"], pre["q_scale"]), "q_scale"
+    assert np.array_equal(V["q_scale"][:, :, :Nq], pre["q_scale"]), "q_scale"
+    assert not V["q_scale"][:, :, Nq:].any(), "q_scale padding"
     nkb = pre["k_scale"].shape[-1]
     assert np.array_equal(V["k_scale"][:, :, :nkb], pre["k_scale"]), "k_scale"
     assert np.array_equal(V["v_scale"], pre["v_scale"]), "v_scale"

@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert sorted(binding.EXPORTED) == names
-    assert L.sage_abi_version() == 3
+    assert L.sage_abi_version() == binding.ABI_VERSION == 4
 
 
 def test_status_strings():

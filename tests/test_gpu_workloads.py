@@ -5,17 +5,17 @@ Pre-pass outputs are compared bit for bit over the whole tensors; the output
 is compared on sampled query tiles (first, last/ragged and random ones) that
 the oracle computes row by row.
 
-Against the mirror: max |diff| <= 2e-2 beyond the effect of FP8 codes of P
-that the exp2 rounding leaves ambiguous (the oracle's `unc`) and beyond half
-an ulp of the 16-bit output type (the store's own rounding: at the x20
-outlier channels outputs reach 16-64, where half a bf16 ulp is 0.0625-0.125),
-and cosine >= 0.9999.  Against exact fp64 attention the GPU must be no worse than the
-method itself (the mirror's own error, +0.002 relative L1 / -0.0005 cosine),
-and within an absolute bound per kind of input: iid inputs 0.06 / 0.998;
-x20 channel outliers in Q/K/V 0.06 / 0.99 (per-block INT8 scales of Q and K
-are dominated by the outlier channels); 2% of tokens x10 0.16 / 0.975 (almost
-every 128-token Q block and 64-token K block holds an outlier token, which
-sets its INT8 scale; the mirror alone measures 0.142 / 0.981 there).
+Against the oracle: max |diff| <= 2e-2 beyond the effect of FP8 codes of P
+that fp32 rounding leaves ambiguous (the oracle's `unc`) and beyond half an
+ulp of the 16-bit output type (the store's own rounding: at the x20 outlier
+channels outputs reach 16-64, where half a bf16 ulp is 0.0625-0.125), and
+cosine >= 0.9999.  Against exact fp64 attention the GPU must be no worse than
+the method itself (the oracle's own error, +0.002 relative L1 / -0.0005
+cosine), and within an absolute bound per kind of input: iid inputs
+0.06 / 0.998; x20 channel outliers in Q/K/V 0.06 / 0.99 (the 32-key K block
+scales are dominated by the outlier channels); 2% of tokens x10
+0.045 / 0.997 (with per-token Q scales and 32-key K blocks the oracle sits
+at the FP8 floor of ~0.031 there).
 """
 import json
 import os
@@ -51,7 +51,7 @@ def test_workload_full_size(name, smooth_k):
     if w.outlier_channels:
         bound = (0.06, 0.99)
     elif w.token_outlier_prob > 0:
-        bound = (0.16, 0.975)
+        bound = (0.045, 0.997)
     else:
         bound = (EXACT_REL_L1, EXACT_COS)
     assert r["rel_l1_exact"] <= bound[0] and r["cos_exact"] >= bound[1], r
