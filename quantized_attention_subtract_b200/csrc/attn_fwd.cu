@@ -13,24 +13,29 @@
 //   out = O * v_scale / l (+ mean_v), rounded to bf16 / fp16
 //
 // One CTA (512 threads, four warpgroups) per SM owns two query tiles, A and
-// B, of one (batch, head), and streams the head's K and V tiles once for both:
-// while one tile's softmax runs, the tensor core works on the other's MMAs.
+// B, of one (batch, head), and streams the head's K and V tiles once for both.
 //   warps 0-3   softmax of tile A, warps 4-7 softmax of tile B: one query row
-//               per thread (TMEM lane); S_j is read with tcgen05.ld, the FP8
-//               P_j is written back into S_j's first 32 columns with
-//               tcgen05.st, and the row's rescale factor goes to shared memory
+//               per thread (TMEM lane).  S_j is read with tcgen05.ld (which
+//               frees S_j's columns for S_{j+1} at once), the row's rescale
+//               factor goes to shared memory, and the FP8 P_j is written to
+//               its own TMEM columns (head dims 64 and 96) or to shared memory
+//               with the 128-byte swizzle (head dim 128, where S and O fill
+//               the 512 TMEM columns).  The two warpgroups take turns for their
+//               exponentials (A's tile j, B's tile j, A's tile j + 1, ...), so
+//               that each has the exp2 units to itself while the other loads
+//               S and takes its max.
 //   warps 8-11  correction: multiply a tile's O rows in TMEM by the rescale
 //               factor (after P V_{j-1}, before P V_j), then the epilogue
-//   warp 12     TMA producer: Q_A, Q_B once, then K_0, V_0, K_1, V_1, ... into
-//               a shared-memory ring (order = MMA consumption order)
-//   warp 13     allocates the 512 TMEM columns and issues the MMAs:
-//               S_A(0), S_B(0), then per KV tile j: O_A += P_A(j) V_j (P from
-//               TMEM), S_A(j+1) once that P V has completed, O_B += P_B(j) V_j,
-//               S_B(j+1); both single-issuer roles run their loop with the
-//               whole warp and issue from one elected lane
+//   warp 12     TMA producer: Q_A, Q_B once, then K_0, K_1, V_0, K_2, V_1, ...
+//               into a shared-memory ring (order = MMA consumption order)
+//   warp 13     allocates the 512 TMEM columns and issues the MMAs, per KV
+//               tile j: S_A(j+1), S_B(j+1) as soon as the softmax warps have
+//               read S(j), then O_A += P_A(j) V_j, O_B += P_B(j) V_j; it runs
+//               its loop with the whole warp and issues from one elected lane
 //   warps 14-15 idle
-// TMEM: S_A at columns [0, 128), S_B at [128, 256), O_A at [256, 256 + D),
-// O_B at [384, 384 + D).
+// TMEM: S_A at columns [0, 128), S_B at [128, 256), O_A and O_B from 256 (D
+// columns each, 128 apart for D = 128), P_A and P_B (32 columns each) after
+// them for D < 128.
 // Causal tiles past the diagonal are skipped; keys >= Nkv and (causal) keys
 // > query are masked; rows >= Nq are computed but not stored.
 // Template flags: smoothed Q (dS added to the logits), variable-length
@@ -56,14 +61,17 @@ template <int D>
 struct Cfg {
   static constexpr int Dp = D == 64 ? 64 : 128;       // INT8 row length in smem / workspace
   static constexpr int kQKSteps = D / 32;             // K = 32 bytes per 8-bit MMA
+  static constexpr bool kPTmem = D < 128;             // FP8 P in TMEM (else shared memory)
   static constexpr int kQBytes = 128 * Dp;
   static constexpr int kKBytes = 128 * Dp;
   static constexpr int kVBytes = D * 128;
+  static constexpr int kPBytes = 128 * 128;           // one tile's P, 128 rows x 128 keys
   static constexpr int kStageBytes = kKBytes > kVBytes ? kKBytes : kVBytes;
   static constexpr int kStages = D == 64 ? 8 : 6;     // 3-4 KV tiles in flight
   static constexpr int kOffQ = 0;                     // Q_A, Q_B
   static constexpr int kOffRing = kOffQ + 2 * kQBytes;
-  static constexpr int kOffBar = kOffRing + kStages * kStageBytes;
+  static constexpr int kOffP = kOffRing + kStages * kStageBytes;  // P_A, P_B (D = 128)
+  static constexpr int kOffBar = kOffP + (kPTmem ? 0 : 2 * kPBytes);
   static constexpr int kBarBytes = 512;
   static constexpr int kOffAlpha = kOffBar + kBarBytes;  // float [2][128] rescale factors
   static constexpr int kOffL = kOffAlpha + 1024;         // float [2][128] row sums
@@ -71,7 +79,15 @@ struct Cfg {
   static constexpr int kSmem = kOffMisc + 64 + 1024;     // +1024: base alignment slack
   static constexpr uint32_t kTmemCols = 512;
   static constexpr int kThreads = 512;
+  // TMEM columns of tile X's S, O and (D < 128) P
+  static __device__ __forceinline__ uint32_t col_s(int X) { return 128u * uint32_t(X); }
+  static __device__ __forceinline__ uint32_t col_o(int X) {
+    return 256u + uint32_t(D == 128 ? 128 : D) * uint32_t(X);
+  }
+  static __device__ __forceinline__ uint32_t col_p(int X) { return 256u + 2u * D + 32u * uint32_t(X); }
 };
+static_assert(256 + 2 * 96 + 64 <= 512 && 256 + 2 * 64 + 64 <= 512, "TMEM columns");
+static_assert(Cfg<128>::kSmem <= 227 * 1024, "shared memory");
 
 // Register split of the attention CTA (512 threads launched at 128 registers
 // each, the whole register file): the helper warpgroup (TMA producer, MMA
@@ -81,23 +97,21 @@ constexpr uint32_t kLaunchRegs = 128, kSoftmaxRegs = 184, kCorrRegs = 96, kHelpe
 static_assert(2 * 128 * kSoftmaxRegs + 128 * kCorrRegs + 128 * kHelperRegs == kLaunchRegs * 512,
               "register split");
 
-// TMEM columns of tile X's S (and P) and O.
-__device__ __forceinline__ uint32_t col_s(int X) { return 128u * uint32_t(X); }
-__device__ __forceinline__ uint32_t col_o(int X) { return 256u + 128u * uint32_t(X); }
-
 // Barrier slots (8 bytes each) inside the barrier area.  [X] = tile A / B.
 enum Bar {
   kBarQ = 0,
   kBarFull = 1,      // + stage (8)   TMA bytes
   kBarEmpty = 9,     // + stage (8)   tcgen05.commit
   kBarSFull = 17,    // + X           tcgen05.commit: S_X(j) in TMEM
-  kBarPReady = 19,   // + X           4 softmax warps: P_X(j) in TMEM, S_X(j) read
-  kBarAlpha = 21,    // + X           4 softmax warps: rescale factors of tile j in smem
-  kBarOReady = 23,   // + X           4 correction warps: O_X ready for P V_j
-  kBarPVDone = 25,   // + X           tcgen05.commit: P V_j of tile X complete
+  kBarSEmpty = 19,   // + X           4 softmax warps: S_X(j) read into registers
+  kBarPReady = 21,   // + X           4 softmax warps: P_X(j) written
+  kBarAlpha = 23,    // + X           4 softmax warps: rescale factors of tile j in smem
+  kBarOReady = 25,   // + X           4 correction warps: O_X ready for P V_j
   kBarLReady = 27,   // + X           4 softmax warps: row sums in smem (once)
-  kBarFinal = 29,
-  kNumBars = 30
+  kBarTurn = 29,     // + X           4 warps of the other softmax warpgroup: X's turn for exp2
+  kBarPVDone = 31,   // + X           tcgen05.commit: P V_j of tile X complete
+  kBarFinal = 33,
+  kNumBars = 34
 };
 static_assert(kNumBars * 8 <= 512, "barrier area");
 
@@ -115,24 +129,26 @@ __device__ __forceinline__ bool warp_wait_h(uint32_t bar, uint32_t parity, int *
 constexpr float kBias = 12582912.0f;  // 1.5 * 2^23
 
 // One query row's share of one KV tile (128 keys), first part: s[] holds the
-// int32 S row from TMEM and is biased in place to the fp32 bit patterns of
-// 1.5 * 2^23 + S (exact for |S| < 2^22, same order as S); with smoothed Q it
-// then holds the logits x = S * c + dsk.  Keys k >= lim (only when kMasked)
-// are set to -inf.  c[q] is the dequantisation factor of keys 32 q .. 32 q +
-// 31.  Returns the tile max of the logits over the valid keys (-inf if none).
+// int32 S row from TMEM.  Without smoothed Q it is converted in place to
+// fp32 (exact: |S| <= 127^2 * 128 < 2^24); with smoothed Q it becomes the
+// logits x = S * c + dsk (S biased to the fp32 bit pattern of 1.5 * 2^23 + S,
+// which is exact, then unbiased in the FMA).  Keys k >= lim (only when
+// kMasked) are set to -inf.  c[q] is the dequantisation factor of keys
+// 32 q .. 32 q + 31.  Returns the tile max of the logits over the valid keys
+// (-inf if none).
 template <bool kMasked, bool kSmoothQ>
 __device__ __forceinline__ float tile_max(uint32_t (&s)[128], const float (&c)[4],
                                           const float *dsk_tile, int lim) {
 #define X(k) __uint_as_float(s[k])
+  if (!kSmoothQ) {
 #pragma unroll
-  for (int k = 0; k < 128; ++k) s[k] += 0x4B400000u;
-  if (kSmoothQ) {
+    for (int k = 0; k < 128; ++k) s[k] = __float_as_uint(__int2float_rn(int(s[k])));
+  } else {
     const float2 nb = make_float2(-kBias, -kBias);
 #pragma unroll
+    for (int k = 0; k < 128; ++k) s[k] += 0x4B400000u;
+#pragma unroll
     for (int k = 0; k < 128; k += 4) {
-      // one 32-key section's dS loads at a time (an empty asm with a memory
-      // clobber keeps the compiler from hoisting all 32 loads)
-      if (k % 32 == 0) asm volatile("" ::: "memory");
       const float4 d4 = __ldg(reinterpret_cast<const float4 *>(dsk_tile + k));
       const float2 c2 = make_float2(c[k / 32], c[k / 32]);
       const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(X(k), X(k + 1)), nb), c2, make_float2(d4.x, d4.y));
@@ -164,27 +180,22 @@ __device__ __forceinline__ float tile_max(uint32_t (&s)[128], const float (&c)[4
 #pragma unroll
   for (int sec = 0; sec < 4; ++sec) {
     const float hs = fmaxf(h[2 * sec], h[2 * sec + 1]);
-    // max_k fl(S_k * c) == fl(max_k S_k * c) since c >= 0; the biased max
-    // minus the bias is max_k S_k exactly
+    // max_k fl(S_k * c) == fl(max_k S_k * c) since c >= 0
     if (kSmoothQ) r = fmaxf(r, hs);
-    else r = fmaxf(r, hs == -INFINITY ? -INFINITY : __fmul_rn(__fsub_rn(hs, kBias), c[sec]));
+    else r = fmaxf(r, hs == -INFINITY ? -INFINITY : __fmul_rn(hs, c[sec]));
   }
   return r;
 #undef X
 }
 
-// Second part: probabilities 2^(x - mb) (mb = m - log2(448), so a key at the
-// row max gets 448), their sum (returned) and their FP8 codes, written to the
-// row's TMEM lane at columns tP .. tP + 31 (keys 4 w .. 4 w + 3 in column w),
-// one 8-column store per 32-key section (issued; the caller waits).  Pairs of
-// keys go through f32x2 ops; every lane of a packed op rounds like its scalar
-// counterpart.
+// The exponent arguments t = x * c - mb (mb = m - log2(448), so a key at the
+// row max gets t = log2(448)), in place, with smoothed Q t = x - mb (x
+// already holds the logit).  Computed before the warpgroup's turn for the
+// exponentials, so that the turn holds only the exp2 and what depends on it.
 template <bool kSmoothQ>
-__device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], const float (&c)[4], float nmb,
-                                          uint32_t tP) {
+__device__ __forceinline__ void tile_args(uint32_t (&s)[128], const float (&c)[4], float nmb) {
 #define X(k) __uint_as_float(s[k])
-  float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
-  const float2 nmb2 = make_float2(nmb, nmb), nb2 = make_float2(-kBias, -kBias);
+  const float2 nmb2 = make_float2(nmb, nmb);
 #pragma unroll
   for (int sec = 0; sec < 4; ++sec) {
     // A scale product of exactly 0 means an all-zero Q row or K block, so
@@ -192,26 +203,47 @@ __device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], const float 
     // and keeps masked keys at -inf * c = -inf instead of NaN.
     const float ce = c[sec] == 0.f ? FLT_MIN : c[sec];
     const float2 c2 = make_float2(ce, ce);
+#pragma unroll
+    for (int k = 32 * sec; k < 32 * sec + 32; k += 2) {
+      const float2 x = make_float2(X(k), X(k + 1));
+      const float2 t = kSmoothQ ? __fadd2_rn(x, nmb2) : __ffma2_rn(x, c2, nmb2);
+      s[k] = __float_as_uint(t.x);
+      s[k + 1] = __float_as_uint(t.y);
+    }
+  }
+#undef X
+}
+
+// Second part: probabilities 2^t of the arguments tile_args left in s[],
+// their sum (returned) and their FP8 codes, stored one 32-key section at a
+// time: kPTmem -- to the row's TMEM lane at columns pdst .. pdst + 31 (keys
+// 4 w .. 4 w + 3 in column w; stores issued, the caller waits); otherwise to
+// the row's 128 bytes of a shared-memory P tile at pdst with the 128-byte
+// swizzle (16-byte unit u at u ^ (row % 8)).  Pairs of keys go through f32x2
+// ops; every lane of a packed op rounds like its scalar counterpart.
+template <bool kPTmem>
+__device__ __forceinline__ float tile_exp(const uint32_t (&s)[128], uint32_t pdst, uint32_t rx) {
+#define X(k) __uint_as_float(s[k])
+  float2 acc01 = make_float2(0.f, 0.f), acc23 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int sec = 0; sec < 4; ++sec) {
     uint32_t pk[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       const int k = 32 * sec + 4 * q;
-      float2 t01, t23;
-      const float2 x01 = make_float2(X(k), X(k + 1)), x23 = make_float2(X(k + 2), X(k + 3));
-      if (kSmoothQ) {
-        t01 = __fadd2_rn(x01, nmb2);
-        t23 = __fadd2_rn(x23, nmb2);
-      } else {
-        t01 = __ffma2_rn(__fadd2_rn(x01, nb2), c2, nmb2);
-        t23 = __ffma2_rn(__fadd2_rn(x23, nb2), c2, nmb2);
-      }
-      const float2 p01 = make_float2(ex2_approx(t01.x), ex2_approx(t01.y));
-      const float2 p23 = make_float2(ex2_approx(t23.x), ex2_approx(t23.y));
+      const float2 p01 = make_float2(ex2_approx(X(k)), ex2_approx(X(k + 1)));
+      const float2 p23 = make_float2(ex2_approx(X(k + 2)), ex2_approx(X(k + 3)));
       acc01 = __fadd2_rn(acc01, p01);
       acc23 = __fadd2_rn(acc23, p23);
       pk[q] = e4m3x4(p01.x, p01.y, p23.x, p23.y);
     }
-    tmem_st8_issue(tP + 8u * uint32_t(sec), pk);
+    if constexpr (kPTmem) {
+      tmem_st8_issue(pdst + 8u * uint32_t(sec), pk);
+    } else {
+      // keys 32 sec .. 32 sec + 31 are the 16-byte units 2 sec and 2 sec + 1 of the row
+      sts128(pdst + ((32u * sec) ^ rx), pk[0], pk[1], pk[2], pk[3]);
+      sts128(pdst + ((32u * sec + 16u) ^ rx), pk[4], pk[5], pk[6], pk[7]);
+    }
   }
   return (acc01.x + acc01.y) + (acc23.x + acc23.y);
 #undef X
@@ -288,6 +320,7 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
   return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+
 template <int D, bool kSmoothQ, bool kVarlen, bool kDump>
 __global__ void __maxnreg__(128)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -300,6 +333,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   // the barrier and TMEM addresses built from them in uniform registers
   const uint32_t s_base = __shfl_sync(0xffffffffu, smem_u32(smem), 0);
   const uint32_t sQ = s_base + C::kOffQ, sRing = s_base + C::kOffRing, bars = s_base + C::kOffBar;
+  const uint32_t sP = s_base + C::kOffP;
   auto bar = [&](int i) { return bars + 8u * uint32_t(i); };
   float *alpha_s = reinterpret_cast<float *>(smem + C::kOffAlpha);
   float *l_s = reinterpret_cast<float *>(smem + C::kOffL);
@@ -339,13 +373,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int T = max(TA, TB);
 
   if (threadIdx.x == 0) {
-    // the softmax warps (4) arrive on P-ready, alpha and L-ready, the
-    // correction warps (4) on O-ready; TMA bytes or a single tcgen05.commit
+    // four warps (of the softmax or correction warpgroups) arrive on the
+    // S-empty ... turn barriers; TMA bytes or a single tcgen05.commit
     // complete the others
-    for (int i = 0; i < kNumBars; ++i) {
-      const bool four = (i >= kBarPReady && i < kBarPVDone) || i == kBarLReady || i == kBarLReady + 1;
-      mbar_init(bar(i), four ? 4 : 1);
-    }
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bar(i), (i >= kBarSEmpty && i < kBarPVDone) ? 4 : 1);
     fence_mbar_init();
     // one read of the status word decides for every warp whether an earlier
     // CTA already failed
@@ -379,28 +410,31 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int n = 0;
       bool ok = true;
       const int krow0 = bhk * ws.Nkv_pad, vrow0 = bhk * D;
-      // K_0, V_0, K_1, V_1, ...
-      for (int j = 0; ok && j < T; ++j) {
-#pragma unroll
-        for (int isV = 0; isV < 2; ++isV) {
-          const int st = n % C::kStages;
-          if (!warp_wait_h(bar(kBarEmpty + st), ((n / C::kStages) & 1) ^ 1, status)) {
-            ok = false;
-            break;
-          }
-          if (leader) {
-            const uint32_t dst = sRing + st * C::kStageBytes, full = bar(kBarFull + st);
-            if (!isV) {
-              mbar_arrive_expect_tx(full, C::kKBytes);
-              tma_load_2d(dst, &tm_k, full, 0, krow0 + j * kKVTile);
-            } else {
-              mbar_arrive_expect_tx(full, C::kVBytes);
-              tma_load_2d(dst, &tm_v, full, j * kKVTile, vrow0);
-            }
-          }
-          __syncwarp();
-          ++n;
+      auto load = [&](bool isV, int j) {
+        if (!ok) return;
+        const int st = n % C::kStages;
+        if (!warp_wait_h(bar(kBarEmpty + st), ((n / C::kStages) & 1) ^ 1, status)) {
+          ok = false;
+          return;
         }
+        if (leader) {
+          const uint32_t dst = sRing + st * C::kStageBytes, full = bar(kBarFull + st);
+          if (!isV) {
+            mbar_arrive_expect_tx(full, C::kKBytes);
+            tma_load_2d(dst, &tm_k, full, 0, krow0 + j * kKVTile);
+          } else {
+            mbar_arrive_expect_tx(full, C::kVBytes);
+            tma_load_2d(dst, &tm_v, full, j * kKVTile, vrow0);
+          }
+        }
+        __syncwarp();
+        ++n;
+      };
+      // K_0, K_1, V_0, K_2, V_1, ..., V_{T-1}
+      load(false, 0);
+      for (int j = 0; ok && j < T; ++j) {
+        if (j + 1 < T) load(false, j + 1);
+        load(true, j);
       }
       // Before leaving, make sure every copy issued has landed (bounded).
       warp_wait_h(bar(kBarQ), 0, status, false);
@@ -420,6 +454,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const uint64_t dQ1 = smem_desc_kmajor(sQ + C::kQBytes, C::Dp);
       const uint64_t dK0 = smem_desc_kmajor(sRing, C::Dp);
       const uint64_t dV0 = smem_desc_kmajor(sRing, 128);
+      const uint64_t dP0 = smem_desc_kmajor(sP, 128);
       int n = 0;
       bool ok = warp_wait_h(bar(kBarQ), 0, status);
       auto wait_stage = [&]() -> uint32_t {
@@ -434,7 +469,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (leader) {
 #pragma unroll
           for (int k = 0; k < C::kQKSteps; ++k)
-            mma_i8_ss(tmem + col_s(X), dQ + 2 * k, dK + 2 * k, id_s, k > 0 ? 1u : 0u);
+            mma_i8_ss(tmem + C::col_s(X), dQ + 2 * k, dK + 2 * k, id_s, k > 0 ? 1u : 0u);
           mma_commit(bar(kBarSFull + X));
         }
         __syncwarp();
@@ -450,46 +485,52 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       for (int j = 0; ok && j < T; ++j) {
-        const uint32_t stV = wait_stage();
-        const bool nextK = j + 1 < T;
-        const uint32_t stK = nextK ? wait_stage() : 0u;
-        if (!ok) break;
+        // S(j+1) of both tiles, each once its softmax warps have read S(j)
+        if (j + 1 < T) {
+          const uint32_t stK = wait_stage();
 #pragma unroll
-        for (int X = 0; X < 2; ++X) {
-          const int TX = X ? TB : TA;
-          if (j >= TX) continue;
-          // P_X(j) written and O_X corrected for tile j
-          if (!warp_wait_h(bar(kBarPReady + X), j & 1, status) ||
-              !warp_wait_h(bar(kBarOReady + X), j & 1, status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t dV = dV0 + stV * kStageStep;
-          if (leader) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_f8_ts(tmem + col_o(X), tmem + col_s(X) + 8u * k, dV + 2 * k, id_o,
-                        (j > 0 || k > 0) ? 1u : 0u);
-            mma_commit(bar(kBarPVDone + X));
-          }
-          __syncwarp();
-          if (j + 1 < TX) {
-            // S_X(j+1) overwrites the columns P_X(j) is read from: wait until
-            // that P V has completed
-            if (!warp_wait_h(bar(kBarPVDone + X), j & 1, status)) {
+          for (int X = 0; X < 2; ++X) {
+            if (!ok || j + 1 >= (X ? TB : TA)) continue;
+            if (!warp_wait_h(bar(kBarSEmpty + X), j & 1, status)) {
               ok = false;
               break;
             }
             tc_fence_after();
             issue_s(X, stK);
           }
+          if (!ok) break;
+          if (leader) mma_commit(bar(kBarEmpty + stK));
+          __syncwarp();
+        }
+        // O_X += P_X(j) V_j once P_X(j) is written and O_X corrected
+        const uint32_t stV = wait_stage();
+        if (!ok) break;
+        const uint64_t dV = dV0 + stV * kStageStep;
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          if (j >= (X ? TB : TA)) continue;
+          if (!warp_wait_h(bar(kBarPReady + X), j & 1, status) ||
+              !warp_wait_h(bar(kBarOReady + X), j & 1, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              if constexpr (C::kPTmem)
+                mma_f8_ts(tmem + C::col_o(X), tmem + C::col_p(X) + 8u * k, dV + 2 * k, id_o,
+                          (j > 0 || k > 0) ? 1u : 0u);
+              else
+                mma_f8_ss(tmem + C::col_o(X), dP0 + uint64_t(X) * (uint64_t(C::kPBytes) >> 4) + 2 * k,
+                          dV + 2 * k, id_o, (j > 0 || k > 0) ? 1u : 0u);
+            }
+            mma_commit(bar(kBarPVDone + X));
+          }
+          __syncwarp();
         }
         if (!ok) break;
-        if (leader) {
-          mma_commit(bar(kBarEmpty + stV));
-          if (nextK) mma_commit(bar(kBarEmpty + stK));
-        }
+        if (leader) mma_commit(bar(kBarEmpty + stV));
         __syncwarp();
       }
       // every MMA issued by the elected lane has finished before teardown
@@ -520,7 +561,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             break;
           }
           tc_fence_after();
-          rescale_row<D>(tmem + lane_off + col_o(X), a);
+          rescale_row<D>(tmem + lane_off + C::col_o(X), a);
           tc_fence_before();
         }
         __syncwarp();
@@ -541,7 +582,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       const int i = (X ? q0B : q0A) + row;
       uint8_t *orow = reinterpret_cast<uint8_t *>(pb.out) +
                       2 * ((kVarlen ? o_off(pb, b) : b * pb.os_b) + h * pb.os_h + (long long)i * pb.os_n);
-      store_row<D>(tmem + lane_off + col_o(X), l_s[X * 128 + row], ws.v_scale + (long long)bhk * D,
+      store_row<D>(tmem + lane_off + C::col_o(X), l_s[X * 128 + row], ws.v_scale + (long long)bhk * D,
                    ws.mean_v + (long long)bhk * D, pb.smooth_v != 0, pb.bf16 != 0, orow, i < Nq_b);
     }
   } else {
@@ -551,7 +592,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int row = 32 * wq + lane;            // row within the query tile (TMEM lane)
     const int q0 = X ? q0B : q0A, TX = X ? TB : TA;
     const int i = q0 + row;                    // query index
-    const uint32_t tS = tmem + (uint32_t(32 * wq) << 16) + col_s(X);
+    const uint32_t lane_off = uint32_t(32 * wq) << 16;
+    const uint32_t tS = tmem + lane_off + C::col_s(X);
+    // where this row's FP8 P goes: its TMEM lane at the tile's P columns, or
+    // its 128 bytes of the tile's shared-memory P buffer (row-major, swizzled)
+    const uint32_t pdst = C::kPTmem ? tmem + lane_off + C::col_p(X)
+                                    : sP + uint32_t(X) * C::kPBytes + uint32_t(row) * 128u;
+    const uint32_t rx = uint32_t(row & 7) << 4;
     if (!skip_all && TX > 0) {
       const float qs = ws.q_scale[(long long)bh * ws.Nq_pad + i];
       const float *ksc = ws.k_scale + (long long)bhk * (ws.Nkv_pad / kKBlk);
@@ -574,6 +621,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_after();
         uint32_t s[128];
         tmem_ld64x2(tS, s);
+        // S_X(j) is in registers: its columns are free for S_X(j + 1)
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(kBarSEmpty + X));
         if constexpr (kDump) {
           if (bh == pb.dump_bh && q0 / kQTile == pb.dump_qt && j == pb.dump_kt)
             for (int k = 0; k < 128; ++k) pb.s_dump[row * 128 + k] = int32_t(s[k]);
@@ -591,16 +642,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // correction warps (1 when the max did not grow)
         const float m_new = fmaxf(m_run, m_tile);
         const float alpha = (m_new > m_run && m_run != -INFINITY) ? ex2_approx(__fsub_rn(m_run, m_new)) : 1.f;
+        // P V_{j-1} has completed: the MMA warp has taken O-ready of tile j - 1,
+        // so the correction warps are done with tile j - 1's factors (the slot
+        // and the alpha / O-ready barrier phases can move on), and P_X(j - 1)
+        // has been read (its buffer can take P_X(j))
+        if (j > 0 && !warp_wait(bar(kBarPVDone + X), (j - 1) & 1, status)) {
+          ok = false;
+          break;
+        }
         alpha_s[X * 128 + row] = alpha;
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kBarAlpha + X));
         m_run = m_new;
         const float nmb = m_run == -INFINITY ? 0.f : -__fsub_rn(m_run, kLog2P8);
-        const float lsum = tile_exp<kSmoothQ>(s, c, nmb, tS);
+        tile_args<kSmoothQ>(s, c, nmb);
+        // The two softmax warpgroups take turns for their exponentials (A's
+        // tile j, B's tile j, A's tile j + 1, ...).
+        if (X == 0 ? (j >= 1 && j - 1 < TB) : (j < TA)) {
+          if (!warp_wait(bar(kBarTurn + X), (X == 0 ? j - 1 : j) & 1, status)) {
+            ok = false;
+            break;
+          }
+        }
+        const float lsum = tile_exp<C::kPTmem>(s, pdst, rx);
+        if (X == 0 ? j < TB : j + 1 < TA) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(kBarTurn + (1 - X)));
+        }
         l = __fmaf_rn(l, alpha, lsum);
-        // the P stores complete, then P_j (and the end of the S_j reads) is
-        // handed to the MMA warp
-        tmem_st_wait();
+        // the P stores complete (TMEM) or become visible to the tensor core's
+        // async proxy (shared memory), then P_j is handed to the MMA warp
+        if constexpr (C::kPTmem) tmem_st_wait();
+        else fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(kBarPReady + X));
