@@ -45,7 +45,9 @@ L2_BYTES = 126 * 1024 * 1024
 # capture per workload.  They describe the kernel built from the sources hashed
 # here; after any change to those sources the traffic is reported as null until
 # it is captured again.
-ATTN_TRAFFIC = {}   # workload name -> {"sources_sha256_16": ..., "bytes": ...}
+ATTN_TRAFFIC = {     # workload name -> {"sources_sha256_16": ..., "bytes": ...}
+    "mha_n4096_d128_bf16": {"sources_sha256_16": "6be216af3e3d4b74", "bytes": 203680256 + 100903680},
+}
 ATTN_SOURCES = ["attn_fwd.cu", "ptx.cuh", "common.cuh"]
 
 
