@@ -47,14 +47,14 @@ L2_BYTES = 126 * 1024 * 1024
 # it is captured again.
 ATTN_TRAFFIC = {     # workload name -> {"sources_sha256_16": ..., "bytes": ...}
     "mha_n4096_d128_bf16": {"sources_sha256_16": "6be216af3e3d4b74", "bytes": 203680256 + 100903680},
+    "gqa_causal_n32768_d128_bf16": {"sources_sha256_16": "6be216af3e3d4b74", "bytes": 496068096 + 221782784},
 }
 ATTN_SOURCES = ["attn_fwd.cu", "ptx.cuh", "common.cuh"]
 
 
 def _prepass_bytes(w: Workload, qd, kd, vd) -> int:
     """Algorithmic bytes of the pre-pass launches of one step: 2 B read and
-    1 B written per element of Q, K and V (the bench runs the pass with the
-    pre-pass quantising Q)."""
+    1 B written per element of Q, K and V."""
     return 3 * (qd.numel() + kd.numel() + vd.numel())
 
 
