@@ -50,7 +50,8 @@ def build(force: bool = False) -> str:
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in
                 ("B", "Hq", "Hkv", "Nq", "Nkv", "D", "layout", "dtype",
-                 "is_causal", "smooth_k", "smooth_q", "smooth_v")] + [("sm_scale", ctypes.c_float)]
+                 "is_causal", "smooth_k", "smooth_q", "smooth_v")] + [("sm_scale", ctypes.c_float),
+                                                                      ("qk_bits", ctypes.c_int)]
 
 
 def _load():
@@ -99,6 +100,7 @@ class Problem:
     smooth_q: bool = False
     smooth_v: bool = False
     sm_scale: float | None = None
+    qk_bits: int = 8         # 8: INT8 Q/K codes in [-127, 127]; 4: INT4 codes in [-7, 7]
 
     def resolved_sm_scale(self) -> np.float32:
         if self.sm_scale is not None and self.sm_scale > 0:
@@ -109,7 +111,7 @@ class Problem:
         return _Params(self.B, self.Hq, self.Hkv, self.Nq, self.Nkv, self.D,
                        0 if self.layout == "HND" else 1, 0 if self.dtype == "fp16" else 1,
                        int(self.is_causal), int(self.smooth_k), int(self.smooth_q),
-                       int(self.smooth_v), float(self.resolved_sm_scale()))
+                       int(self.smooth_v), float(self.resolved_sm_scale()), int(self.qk_bits))
 
     @property
     def nqb(self) -> int:

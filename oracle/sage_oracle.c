@@ -33,6 +33,10 @@
  *     code = rint(x * (127/amax)) with round-half-even, computed in IEEE
  *     fp32 without FMA contraction.  A block with amax < 2^-64 gets scale 0
  *     and all-zero codes.
+ *   - The 4-bit variant (SageAttention2 technical report, section 1: Q and
+ *     K in INT4 at warp level; section 3: 8 bits for the sensitive layers,
+ *     4 bits elsewhere) uses the same blocks with codes in [-7, 7]:
+ *     scale = amax/7, code = rint(x * (7/amax)).
  *   - Means are exact fixed-point means: sum of rint(x * 2^24) in int64,
  *     divided in fp64 by n * 2^24 and rounded to fp32.  This makes the mean
  *     independent of summation order.  Q's smoothing mean is taken per block
@@ -74,6 +78,7 @@ typedef struct {
     int dtype;       /* 0 = fp16, 1 = bf16 */
     int is_causal, smooth_k, smooth_q, smooth_v;
     float sm_scale;  /* already resolved (> 0) */
+    int qk_bits;     /* 8: INT8 codes of Q and K in [-127, 127]; 4: INT4 codes in [-7, 7] */
 } oracle_params;
 
 int oracle_num_threads(void) {
@@ -192,8 +197,9 @@ static float fixed_point_mean(const double *x, int64_t n) {
     return (float)((double)acc / ((double)n * 16777216.0));
 }
 
-/* Symmetric INT8 quantisation of one block (fp32 arithmetic). */
-static float quantise_int8_block(const float *x, int64_t n, int8_t *codes) {
+/* Symmetric integer quantisation of one block (fp32 arithmetic): codes in
+ * [-qmax, qmax], qmax = 127 (INT8) or 7 (INT4). */
+static float quantise_int_block(const float *x, int64_t n, int8_t *codes, float qmax) {
     float amax = 0.0f;
     for (int64_t i = 0; i < n; i++) {
         float a = fabsf(x[i]);
@@ -203,13 +209,13 @@ static float quantise_int8_block(const float *x, int64_t n, int8_t *codes) {
         for (int64_t i = 0; i < n; i++) codes[i] = 0;
         return 0.0f;
     }
-    float scale = amax / 127.0f;
-    float inv = 127.0f / amax;
+    float scale = amax / qmax;
+    float inv = qmax / amax;
     for (int64_t i = 0; i < n; i++) {
         float t = x[i] * inv;
         float r = nearbyintf(t);
-        if (r > 127.0f) r = 127.0f;
-        if (r < -127.0f) r = -127.0f;
+        if (r > qmax) r = qmax;
+        if (r < -qmax) r = -qmax;
         codes[i] = (int8_t)r;
     }
     return scale;
@@ -236,6 +242,8 @@ void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k
     const int D = p->D, Nq = p->Nq, Nkv = p->Nkv;
     const int nmb = (Nq + QMBLK - 1) / QMBLK, nkb = (Nkv + KBLK - 1) / KBLK;
 
+    const float qmax = p->qk_bits == 4 ? 7.0f : 127.0f;
+
     /* K: mean over all tokens, K' = K - mean, per-32-token INT8 blocks. */
 #pragma omp parallel for collapse(2) schedule(dynamic)
     for (int b = 0; b < p->B; b++)
@@ -250,9 +258,9 @@ void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k
             }
             for (int kb = 0; kb < nkb; kb++) {
                 int j0 = kb * KBLK, n = (Nkv - j0 < KBLK) ? Nkv - j0 : KBLK;
-                k_scale[((int64_t)b * p->Hkv + h) * nkb + kb] = quantise_int8_block(
+                k_scale[((int64_t)b * p->Hkv + h) * nkb + kb] = quantise_int_block(
                     kph + (int64_t)j0 * D, (int64_t)n * D,
-                    k8 + (((int64_t)b * p->Hkv + h) * Nkv + j0) * D);
+                    k8 + (((int64_t)b * p->Hkv + h) * Nkv + j0) * D, qmax);
             }
             free(col);
         }
@@ -274,7 +282,7 @@ void oracle_prepass(const oracle_params *p, const uint16_t *q, const uint16_t *k
                 }
                 for (int r = 0; r < n; r++) {
                     const int64_t row = ((int64_t)b * p->Hq + h) * Nq + i0 + r;
-                    q_scale[row] = quantise_int8_block(blk + (int64_t)r * D, D, q8 + row * D);
+                    q_scale[row] = quantise_int_block(blk + (int64_t)r * D, D, q8 + row * D, qmax);
                     if (qp) memcpy(qp + row * D, blk + (int64_t)r * D, sizeof(float) * (size_t)D);
                 }
             }
