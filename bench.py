@@ -1,6 +1,7 @@
 """Benchmark of the quantized attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--qk-bits 8|4] [--varlen] [--no-cpu-baseline]
 
 A step is one whole pass (smoothing + quantisation pre-pass, then the
 attention kernel) over one batch of the named synthetic workload (default:
@@ -129,7 +130,7 @@ def _oracle_problem(w: Workload):
     import oracle
     return oracle.Problem(B=w.B, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, Nkv=w.Nkv, D=w.D, layout=w.layout,
                           dtype=w.dtype, is_causal=w.is_causal, smooth_k=w.smooth_k,
-                          smooth_q=w.smooth_q, smooth_v=w.smooth_v)
+                          smooth_q=w.smooth_q, smooth_v=w.smooth_v, qk_bits=w.qk_bits)
 
 
 def oracle_sample(w: Workload, kv_heads: int, q_tiles: int | None = None):
@@ -264,7 +265,8 @@ def run_reference(args, w: Workload):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "i8xi8->i64 (QK), e4m3xe4m3->f64 (PV)", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nkv": w.Nkv,
-                   "D": w.D, "layout": w.layout, "causal": w.is_causal, "smooth_k": w.smooth_k},
+                   "D": w.D, "layout": w.layout, "causal": w.is_causal, "smooth_k": w.smooth_k,
+                   "qk_bits": w.qk_bits},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -292,7 +294,7 @@ def run_ours(args, w: Workload):
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     out = torch.empty_like(qd)
     p = binding.make_params(qd, kd, vd, out, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q,
-                            w.smooth_v)
+                            w.smooth_v, qk_bits=w.qk_bits)
     ws = binding.alloc_workspace(p, dev)
     stream = torch.cuda.current_stream(dev)
     in_bytes = qd.numel() * 2 + kd.numel() * 2 + vd.numel() * 2
@@ -341,13 +343,15 @@ def run_ours(args, w: Workload):
     qh, kh, vh = (x.cpu().pin_memory() for x in (qd, kd, vd))
     oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
     for _ in range(2):
-        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh)
+        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh,
+                 qk_bits=w.qk_bits)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(3, min(args.steps, 10))
     e0.record(stream)
     for _ in range(e2e_steps):
-        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh)
+        sageattn(qh, kh, vh, w.layout, w.is_causal, None, w.smooth_k, w.smooth_q, w.smooth_v, out=oh,
+                 qk_bits=w.qk_bits)
     e1.record(stream)
     barrier()
     e2e_ms, = max_over_ranks([e0.elapsed_time(e1) / e2e_steps], pg, dev)
@@ -362,11 +366,12 @@ def run_ours(args, w: Workload):
     line = {
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "i8xi8->i32 (QK), e4m3xe4m3->f32 (PV)",
+        "vs_baseline": None,
+        "dtype": ("i8xi8->i32 (QK)" if w.qk_bits == 8 else "i4 codes in i8xi8->i32 (QK)") + ", e4m3xe4m3->f32 (PV)",
         "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nkv": w.Nkv,
                    "D": w.D, "layout": w.layout, "input_dtype": w.dtype, "causal": w.is_causal,
-                   "smooth_k": w.smooth_k, "parallelism": f"replicas x{world}",
+                   "smooth_k": w.smooth_k, "qk_bits": w.qk_bits, "parallelism": f"replicas x{world}",
                    "l2": f"inputs {in_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)"},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel", "achieved": achieved,
                      "peak": peak8, "unit": "TFLOP/s", "frac": achieved / peak8, "traffic": _attn_traffic(w),
@@ -507,10 +512,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--varlen", action="store_true",
                     help="time the variable-length batch instead of --workload (one GPU)")
+    ap.add_argument("--qk-bits", type=int, default=8, choices=[8, 4],
+                    help="bits of the Q and K codes (4: the INT4 variant)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = WORKLOADS[args.workload]
+    w = WORKLOADS[args.workload].with_(qk_bits=args.qk_bits)
     if args.varlen and args.impl == "ours":
         run_varlen(args)
         return

@@ -15,7 +15,10 @@
  *   2. quantisation: symmetric INT8 Q with one fp32 scale per token and K
  *      with one per block of 32 tokens (the pages' per-block / per-thread
  *      granularity: closerAI blog, part 4; "SageAttention2: Technical
- *      report", section 1); V to FP8 e4m3 with per-channel scales;
+ *      report", section 1); V to FP8 e4m3 with per-channel scales.  On
+ *      request (qk_bits = 4) Q and K take INT4 codes in [-7, 7] on the same
+ *      blocks instead: the report's 4-bit variant (section 1), which its
+ *      section 3 applies to all but the most sensitive layers;
  *   3. a flash-style kernel: INT8 Q K^T with exact int32 accumulation,
  *      dequantisation, online softmax in base 2 with the row's running max
  *      m raised to every 128-key tile's max and the running sum rescaled
@@ -51,7 +54,7 @@
 extern "C" {
 #endif
 
-#define SAGE_ABI_VERSION 4
+#define SAGE_ABI_VERSION 5
 
 /* A CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
 typedef struct CUstream_st *sage_stream_t;
@@ -113,6 +116,12 @@ typedef struct {
    * scales; causal masking top-left within it).  The arrays are copied
    * during the call. */
   const int32_t *cu_seqlens_q, *cu_seqlens_kv;
+  /* Bits of the Q and K codes: 8 (or 0) for INT8 codes in [-127, 127], 4 for
+   * INT4 codes in [-7, 7] (scale = amax / 7 per block).  INT4 codes are held
+   * in the same int8 workspace buffers and multiplied on the INT8 tensor
+   * path, which computes their products exactly; V and P stay FP8.  Any
+   * other value is SAGE_ERR_INVALID_ARG. */
+  int32_t qk_bits;
 } sage_attn_params_t;
 
 /* Where the quantised tensors live inside the workspace (tests, debugging).
@@ -120,8 +129,8 @@ typedef struct {
  * INT8 row length Dp is 64 for D = 64 and 128 otherwise (zero padded).
  * Padding rows and columns hold zero codes. */
 typedef struct {
-  int8_t *q8;        /* [B*Hq ][Nq_pad ][Dp]  INT8 codes of Q (or Q - mq)       */
-  int8_t *k8;        /* [B*Hkv][Nkv_pad][Dp]  INT8 codes of K - mean_k           */
+  int8_t *q8;        /* [B*Hq ][Nq_pad ][Dp]  INT8 (or INT4) codes of Q (or Q - mq) */
+  int8_t *k8;        /* [B*Hkv][Nkv_pad][Dp]  INT8 (or INT4) codes of K - mean_k */
   uint8_t *v8t;      /* [B*Hkv][D][Nkv_pad]   FP8 e4m3 codes of V (- mean_v), transposed */
   float *q_scale;    /* [B*Hq ][Nq_pad]       one per query token (0 past Nq)    */
   float *k_scale;    /* [B*Hkv][Nkv_pad/32]   one per 32 keys                    */

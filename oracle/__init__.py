@@ -289,7 +289,7 @@ def varlen_attention(Hq: int, Hkv: int, D: int, cu_q, cu_kv, q: np.ndarray, k: n
                      v: np.ndarray, dtype: str = "fp16", is_causal: bool = False,
                      smooth_k: bool = True, smooth_q: bool = False, smooth_v: bool = False,
                      sm_scale: float | None = None, with_uncertainty: bool = False,
-                     exact: bool = False) -> dict:
+                     exact: bool = False, qk_bits: int = 8) -> dict:
     """A variable-length batch of packed sequences ("variable sequence lengths
     per batch", sageattention package page): sequence b is rows
     cu_q[b] .. cu_q[b+1] of q [total_q, Hq, D] attending to rows
@@ -312,7 +312,7 @@ def varlen_attention(Hq: int, Hkv: int, D: int, cu_q, cu_kv, q: np.ndarray, k: n
         q0, q1, k0, k1 = int(cu_q[b]), int(cu_q[b + 1]), int(cu_kv[b]), int(cu_kv[b + 1])
         pr = Problem(B=1, Hq=Hq, Hkv=Hkv, Nq=q1 - q0, Nkv=k1 - k0, D=D, layout="NHD", dtype=dtype,
                      is_causal=is_causal, smooth_k=smooth_k, smooth_q=smooth_q, smooth_v=smooth_v,
-                     sm_scale=sm_scale)
+                     sm_scale=sm_scale, qk_bits=qk_bits)
         res["problems"].append(pr)
         if q1 == q0:
             res["pre"].append(None)

@@ -29,7 +29,7 @@ EXPORTED = ["sage_abi_version", "sage_status_string", "sage_workspace_size", "sa
             "sage_debug_wait_timeout", "sage_get_device_status", "sage_attn_fwd_noalloc",
             "sage_noalloc_device_status", "sage_attn_fwd_prepass", "sage_attn_fwd_attention"]
 
-ABI_VERSION = 4
+ABI_VERSION = 5
 
 
 class SageError(RuntimeError):
@@ -53,6 +53,7 @@ class Params(ctypes.Structure):
         ("sm_scale", ctypes.c_float),
         ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
         ("cu_seqlens_q", ctypes.c_void_p), ("cu_seqlens_kv", ctypes.c_void_p),
+        ("qk_bits", ctypes.c_int32),
     ]
 
 
@@ -138,8 +139,9 @@ def _dims(x: torch.Tensor, layout: str):
 
 
 def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scale=None,
-                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None) -> Params:
-    """Fill sage_attn_params_t from torch tensors (no copies, strides as given)."""
+                smooth_k=True, smooth_q=False, smooth_v=False, workspace=None, qk_bits=8) -> Params:
+    """Fill sage_attn_params_t from torch tensors (no copies, strides as given).
+    qk_bits: 8 (INT8 Q and K codes) or 4 (INT4 codes in [-7, 7])."""
     B, Hq, Nq, D = _dims(q, tensor_layout)
     Bk, Hkv, Nkv, Dk = _dims(k, tensor_layout)
     if v.shape != k.shape:
@@ -160,6 +162,7 @@ def make_params(q, k, v, out=None, tensor_layout="HND", is_causal=False, sm_scal
     p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
                                                        int(bool(smooth_q)), int(bool(smooth_v)))
     p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
+    p.qk_bits = int(qk_bits)
     if workspace is not None:
         p.workspace, p.workspace_bytes = workspace.data_ptr(), workspace.numel()
     return p
@@ -177,7 +180,7 @@ def _host_offsets(cu) -> np.ndarray:
 
 def make_varlen_params(q, k, v, out, cu_seqlens_q, cu_seqlens_kv, max_seqlen_q=None,
                        max_seqlen_kv=None, is_causal=False, sm_scale=None, smooth_k=True,
-                       smooth_q=False, smooth_v=False, workspace=None) -> Params:
+                       smooth_q=False, smooth_v=False, workspace=None, qk_bits=8) -> Params:
     """sage_attn_params_t for a variable-length batch: q [total_q, Hq, D],
     k, v [total_kv, Hkv, D] (packed sequences), out like q; cu_seqlens_* hold
     B + 1 offsets (host or device integer tensors / arrays, copied to host
@@ -207,6 +210,7 @@ def make_varlen_params(q, k, v, out, cu_seqlens_q, cu_seqlens_kv, max_seqlen_q=N
     p.is_causal, p.smooth_k, p.smooth_q, p.smooth_v = (int(bool(is_causal)), int(bool(smooth_k)),
                                                        int(bool(smooth_q)), int(bool(smooth_v)))
     p.sm_scale = float(sm_scale) if sm_scale is not None else 0.0
+    p.qk_bits = int(qk_bits)
     p.cu_seqlens_q, p.cu_seqlens_kv = cq.ctypes.data, ck.ctypes.data
     p._offsets = (cq, ck)  # the arrays must outlive every call made with p
     if workspace is not None:
@@ -218,17 +222,17 @@ def sageattn_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlen
                     max_seqlen_q: int | None = None, max_seqlen_k: int | None = None,
                     is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
                     smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
-                    workspace: torch.Tensor | None = None) -> torch.Tensor:
+                    workspace: torch.Tensor | None = None, qk_bits: int = 8) -> torch.Tensor:
     """Quantized attention over a variable-length batch of packed sequences on
     the current CUDA stream: q [total_q, Hq, D], k, v [total_kv, Hkv, D] on
     the device; sequence b owns tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]
     of q (cu_seqlens_k of k, v) and attends only within itself.  Returns out
-    shaped like q."""
+    shaped like q.  qk_bits as in sageattn."""
     if not (q.is_cuda and k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be CUDA tensors")
     dev_out = torch.empty_like(q) if out is None else out
     p = make_varlen_params(q, k, v, dev_out, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                           is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+                           is_causal, sm_scale, smooth_k, smooth_q, smooth_v, qk_bits=qk_bits)
     ws = workspace if workspace is not None else alloc_workspace(p, q.device)
     if workspace is not None:
         p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
@@ -252,10 +256,13 @@ def alloc_workspace(p: Params, device) -> torch.Tensor:
 def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: str = "HND",
              is_causal: bool = False, sm_scale: float | None = None, smooth_k: bool = True,
              smooth_q: bool = False, smooth_v: bool = False, out: torch.Tensor | None = None,
-             workspace: torch.Tensor | None = None) -> torch.Tensor:
+             workspace: torch.Tensor | None = None, qk_bits: int = 8) -> torch.Tensor:
     """Quantized attention forward: INT8 Q K^T, FP8 P V, on the current CUDA stream.
 
     q: [B, Hq, Nq, D] ("HND") or [B, Nq, Hq, D] ("NHD"); k, v: same with Hkv, Nkv.
+    qk_bits=4 selects the 4-bit variant: INT4 codes of Q and K in [-7, 7] on
+    the same blocks (one scale per query token, one per 32 keys), for the
+    layers that tolerate it; 8 keeps INT8.
     Host (CPU) tensors are moved to the current device and the result back, in
     chunks of whole (batch, kv-head group) slices so that the host-to-device
     copy of one chunk, the kernels of the previous one and the device-to-host
@@ -265,12 +272,12 @@ def sageattn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, tensor_layout: s
     """
     if not q.is_cuda:
         return _sageattn_host(q, k, v, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                              smooth_v, out)
+                              smooth_v, out, qk_bits)
     if not (k.is_cuda and v.is_cuda):
         raise ValueError("q, k, v must be on the same device")
     dev_out = torch.empty_like(q) if out is None else out
     p = make_params(q, k, v, dev_out, tensor_layout, is_causal, sm_scale, smooth_k, smooth_q,
-                    smooth_v)
+                    smooth_v, qk_bits=qk_bits)
     if workspace is None:
         workspace = alloc_workspace(p, q.device)
     else:
@@ -303,7 +310,7 @@ def _host_chunks(B: int, Hkv: int, group: int, bytes_per_kv_head: int, layout: s
     return chunks
 
 
-def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out):
+def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, out, qk_bits=8):
     dev = torch.device("cuda", torch.cuda.current_device())
     B, Hq, Nq, D = _dims(q, layout)
     _, Hkv, Nkv, _ = _dims(k, layout)
@@ -327,7 +334,7 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
     first = make_params(sl(qd, *chunks[0][:1], chunks[0][1] * group, chunks[0][2] * group),
                         sl(kd, *chunks[0]), sl(vd, *chunks[0]),
                         sl(od, chunks[0][0], chunks[0][1] * group, chunks[0][2] * group),
-                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+                        layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v, qk_bits=qk_bits)
     ws = alloc_workspace(first, dev)
     done_out = None
     for b, h0, h1 in chunks:
@@ -341,7 +348,8 @@ def _sageattn_host(q, k, v, layout, is_causal, sm_scale, smooth_k, smooth_q, smo
             landed = torch.cuda.Event()
             landed.record(h2d)
         compute.wait_event(landed)
-        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v)
+        p = make_params(qc, kc, vc, oc, layout, is_causal, sm_scale, smooth_k, smooth_q, smooth_v,
+                        qk_bits=qk_bits)
         need = workspace_bytes(p)
         if need > ws.numel():
             ws = torch.empty(need, dtype=torch.uint8, device=dev)

@@ -56,10 +56,8 @@ struct Problem {
   int is_causal, smooth_k, smooth_q, smooth_v;
   float sm_scale;
   float K2;  // fp32(sm_scale * fp32(log2 e))
-  // Q quantised inside the attention kernel (from the 16-bit input, through a
-  // 4-D tensor map) instead of by the pre-pass; the pre-pass then skips Q.
-  int q_fused;
-  int q_map_hn;  // tensor-map dimension order (D, Hq, Nq, B) instead of (D, Nq, Hq, B)
+  // largest code of the Q and K quantisation: 127 (INT8) or 7 (INT4)
+  float qmax;
   // Variable-length batches: batch entry b is sequence b with tokens
   // [cu_q[b], cu_q[b+1]) of the packed q (and cu_kv of k, v); Nq / Nkv are
   // then the maximum lengths and the batch strides are unused.  Null for

@@ -388,14 +388,15 @@ __device__ __forceinline__ void store_codes(uint8_t *dst, int Dp, int c8, int rg
   }
 }
 
-// INT8 scale and reciprocal of a block with absolute maximum a (IEEE fp32
-// divisions): scale = a / 127, inv = 127 / a; both 0 below kTinyAmax.
-__device__ __forceinline__ void int8_scale(float a, float &scale, float &inv) {
+// Integer scale and reciprocal of a block with absolute maximum a (IEEE fp32
+// divisions): scale = a / qmax, inv = qmax / a (qmax = 127 for INT8 codes, 7
+// for INT4); both 0 below kTinyAmax.
+__device__ __forceinline__ void int_scale(float a, float qmax, float &scale, float &inv) {
   scale = 0.f;
   inv = 0.f;
   if (a >= kTinyAmax) {
-    scale = __fdiv_rn(a, 127.0f);
-    inv = __fdiv_rn(127.0f, a);
+    scale = __fdiv_rn(a, qmax);
+    inv = __fdiv_rn(qmax, a);
   }
 }
 
@@ -421,14 +422,12 @@ struct QUnit {
   long long stride;
 };
 
-// Units of quantize_kernel: K and V tiles (both), then Q tiles unless the
-// attention kernel quantises Q; variable-length batches count only the tiles
-// inside a sequence.
+// Units of quantize_kernel: K and V tiles (both), then Q tiles; variable-length
+// batches count only the tiles inside a sequence.
 __host__ __device__ __forceinline__ long long quant_units(const Problem &pb, const Workspace &ws) {
   const long long nKV = pb.cu_kv ? (long long)pb.Hkv * pb.tot_kv128
                                  : (long long)pb.B * pb.Hkv * (ws.Nkv_pad / kKVTile);
-  const long long nQ = pb.q_fused ? 0LL : pb.cu_q ? (long long)pb.Hq * pb.tot_q128
-                                                  : (long long)pb.B * pb.Hq * ws.nqb;
+  const long long nQ = pb.cu_q ? (long long)pb.Hq * pb.tot_q128 : (long long)pb.B * pb.Hq * ws.nqb;
   return 2 * nKV + nQ;
 }
 
@@ -601,11 +600,11 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       if ((threadIdx.x & 31) == 0) atomicMax(mx + rg / 8, __float_as_uint(a));
       __syncthreads();
       float inv[4], sc;
-      int8_scale(__uint_as_float(mx[rg / 8]), sc, inv[0]);
+      int_scale(__uint_as_float(mx[rg / 8]), pb.qmax, sc, inv[0]);
       inv[1] = inv[2] = inv[3] = inv[0];
       if (threadIdx.x < 4) {
         float s4, i4;
-        int8_scale(__uint_as_float(mx[threadIdx.x]), s4, i4);
+        int_scale(__uint_as_float(mx[threadIdx.x]), pb.qmax, s4, i4);
         ws.k_scale[(long long)q.bh * (ws.Nkv_pad / kKBlk) + 4 * q.t + threadIdx.x] = s4;
       }
       store_codes(reinterpret_cast<uint8_t *>(ws.k8) + ((long long)q.bh * ws.Nkv_pad + q.r0) * Dp, Dp,
@@ -704,7 +703,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
 #pragma unroll
         for (int r = 0; r < 4; ++r) a[r] = fmaxf(a[r], __shfl_xor_sync(0xffffffffu, a[r], o));
 #pragma unroll
-      for (int r = 0; r < 4; ++r) int8_scale(a[r], sc[r], inv[r]);
+      for (int r = 0; r < 4; ++r) int_scale(a[r], pb.qmax, sc[r], inv[r]);
       if (c8 < 4) {
         // lane c8 of the group stores row 4 rg + c8's scale (0 past nvalid)
         const float s = c8 == 0 ? sc[0] : c8 == 1 ? sc[1] : c8 == 2 ? sc[2] : sc[3];

@@ -47,6 +47,7 @@ sage_status_t check_shape(const sage_attn_params_t *p) {
       !is_flag(p->smooth_v))
     return SAGE_ERR_INVALID_ARG;
   if (!(p->sm_scale == p->sm_scale) || std::isinf(p->sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (p->qk_bits != 0 && p->qk_bits != 8 && p->qk_bits != 4) return SAGE_ERR_INVALID_ARG;
   // TMA row coordinates and kernel indices are 32-bit
   const long long nq_pad = (p->Nq + 127LL) / 128 * 128, nkv_pad = (p->Nkv + 127LL) / 128 * 128;
   if ((long long)p->B * p->Hq * nq_pad >= (1LL << 31)) return SAGE_ERR_UNSUPPORTED;
@@ -214,6 +215,7 @@ Problem make_problem(const sage_attn_params_t *p) {
   pb.sm_scale = p->sm_scale > 0.f ? p->sm_scale : 1.0f / std::sqrt(float(p->D));
   volatile float l2e = kLog2e;  // keep the product a single fp32 rounding
   pb.K2 = pb.sm_scale * l2e;
+  pb.qmax = p->qk_bits == 4 ? 7.0f : 127.0f;
   return pb;
 }
 

@@ -53,6 +53,7 @@ class Workload:
     token_outlier_prob: float = 0.0
     token_outlier_scale: float = 1.0
     seed: int = 0
+    qk_bits: int = 8          # bits of the Q and K codes the pass is run with (8 or 4)
 
     @property
     def ops(self) -> float:

@@ -24,7 +24,7 @@ EXACT_COS = 0.998
 def oracle_problem(w: Workload) -> oracle.Problem:
     return oracle.Problem(B=w.B, Hq=w.Hq, Hkv=w.Hkv, Nq=w.Nq, Nkv=w.Nkv, D=w.D, layout=w.layout,
                           dtype=w.dtype, is_causal=w.is_causal, smooth_k=w.smooth_k,
-                          smooth_q=w.smooth_q, smooth_v=w.smooth_v)
+                          smooth_q=w.smooth_q, smooth_v=w.smooth_v, qk_bits=w.qk_bits)
 
 
 def to_device(bits: np.ndarray, dtype: str, device="cuda") -> torch.Tensor:
@@ -40,7 +40,7 @@ class DeviceRun:
         self.q, self.k, self.v = (to_device(x, w.dtype) for x in (q, k, v))
         self.out = torch.empty_like(self.q)
         self.p = binding.make_params(self.q, self.k, self.v, self.out, w.layout, w.is_causal, None,
-                                     w.smooth_k, w.smooth_q, w.smooth_v)
+                                     w.smooth_k, w.smooth_q, w.smooth_v, qk_bits=w.qk_bits)
         self.ws = binding.alloc_workspace(self.p, self.q.device)
         if run_attention:
             binding.attn_fwd(self.p, self.q.device)

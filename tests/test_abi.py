@@ -25,7 +25,7 @@ def test_library_exports_every_declared_symbol():
     for n in names:
         assert hasattr(L, n), n
     assert sorted(binding.EXPORTED) == names
-    assert L.sage_abi_version() == binding.ABI_VERSION == 4
+    assert L.sage_abi_version() == binding.ABI_VERSION == 5
 
 
 def test_status_strings():
@@ -48,6 +48,16 @@ def _params(**kw):
 def _ws_size(p):
     n = ctypes.c_size_t(0)
     return binding.lib().sage_workspace_size(ctypes.byref(p), ctypes.byref(n)), n.value
+
+
+@pytest.mark.parametrize("bits,ok", [(0, True), (8, True), (4, True), (1, False), (5, False),
+                                     (16, False), (-4, False)])
+def test_qk_bits_values(bits, ok):
+    st, n = _ws_size(_params(qk_bits=bits))
+    assert (st == 0) == ok
+    if ok:
+        # the 4-bit codes live in the same buffers: same workspace size
+        assert n == _ws_size(_params())[1]
 
 
 def _contract():
