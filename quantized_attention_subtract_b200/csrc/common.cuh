@@ -108,9 +108,9 @@ __device__ __forceinline__ void seq_unit(const int *pc, int B, int heads, long l
                                          int &t) {
   b = seq_of(pc, B, heads, x);
   const int n = pc[b + 1] - pc[b];
-  const long long r = x - (long long)pc[b] * heads;
-  h = int(r / n);
-  t = int(r % n);
+  const int r = int(x - (long long)pc[b] * heads);  // unit counts stay below 2^31
+  h = r / n;
+  t = r % n;
 }
 
 // Per batch entry: query / key counts, and the element offset of (token 0,

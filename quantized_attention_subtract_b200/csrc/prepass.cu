@@ -188,8 +188,10 @@ __global__ void __launch_bounds__(256, 2) kv_stats_kernel(Problem pb, Workspace 
       bh = b * pb.Hkv + h;
       j0 = t * kStatChunk;
     } else {
-      bh = int(u / nchunk);
-      j0 = int(u % nchunk) * kStatChunk;
+      // unit counts stay below 2^31 (the host's size checks): 32-bit division
+      const int ui = int(u);
+      bh = ui / nchunk;
+      j0 = (ui % nchunk) * kStatChunk;
     }
     n = min(kStatChunk, nkv_of(pb, bh / pb.Hkv) - j0);  // <= 0: past this sequence's end
   };
@@ -449,14 +451,14 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
   const long long nKV = kVarlen ? (long long)pb.Hkv * pb.tot_kv128 : (long long)pb.B * pb.Hkv * nKt;
   if (u < 2 * nKV) {
     q.kind = int(u & 1);
-    const long long kvi = nKV - 1 - (u >> 1);  // reverse head order
+    const int kvi = int(nKV - 1 - (u >> 1));  // reverse head order (counts < 2^31)
     if (kVarlen) {
       const int2 bt = seq_unit_ht(pb.pc_kv128, pb.B, pb.Hkv, kvi);
       q.bh = bt.x;
       q.t = bt.y;
     } else {
-      q.t = int(kvi % nKt);
-      q.bh = int(kvi / nKt);
+      q.t = kvi % nKt;
+      q.bh = kvi / nKt;
     }
     q.b = q.bh / pb.Hkv;
     q.h = q.bh % pb.Hkv;
@@ -470,15 +472,15 @@ __device__ __forceinline__ QUnit quant_unit(const Problem &pb, const Workspace &
       q.stride = pb.vs_n;
     }
   } else {
-    const long long qi = u - 2 * nKV;
+    const int qi = int(u - 2 * nKV);
     q.kind = 2;
     if (kVarlen) {
       const int2 bt = seq_unit_ht(pb.pc_q128, pb.B, pb.Hq, qi);
       q.bh = bt.x;
       q.t = bt.y;
     } else {
-      q.t = int(qi % ws.nqb);
-      q.bh = int(qi / ws.nqb);
+      q.t = qi % ws.nqb;
+      q.bh = qi / ws.nqb;
     }
     q.b = q.bh / pb.Hq;
     q.h = q.bh % pb.Hq;
@@ -690,7 +692,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
               for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], chan[8 * c8 + e]);
         }
       }
-      float a[4], inv[4], sc[4];
+      float a[4], inv[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         a[r] = 0.f;
@@ -702,13 +704,15 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       for (int o = L / 2; o > 0; o >>= 1)
 #pragma unroll
         for (int r = 0; r < 4; ++r) a[r] = fmaxf(a[r], __shfl_xor_sync(0xffffffffu, a[r], o));
+      // lane c8 < 4 of the group divides for row 4 rg + c8 (IEEE divisions)
+      // and stores its scale (0 past nvalid); the group's lanes take the four
+      // reciprocals by shuffles
+      float s_own, i_own;
+      int_scale(c8 == 0 ? a[0] : c8 == 1 ? a[1] : c8 == 2 ? a[2] : a[3], pb.qmax, s_own, i_own);
+      const int gbase = int(threadIdx.x & 31) & ~(L - 1);
 #pragma unroll
-      for (int r = 0; r < 4; ++r) int_scale(a[r], pb.qmax, sc[r], inv[r]);
-      if (c8 < 4) {
-        // lane c8 of the group stores row 4 rg + c8's scale (0 past nvalid)
-        const float s = c8 == 0 ? sc[0] : c8 == 1 ? sc[1] : c8 == 2 ? sc[2] : sc[3];
-        ws.q_scale[(long long)q.bh * ws.Nq_pad + q.r0 + 4 * rg + c8] = s;
-      }
+      for (int r = 0; r < 4; ++r) inv[r] = __shfl_sync(0xffffffffu, i_own, gbase + r);
+      if (c8 < 4) ws.q_scale[(long long)q.bh * ws.Nq_pad + q.r0 + 4 * rg + c8] = s_own;
       store_codes(reinterpret_cast<uint8_t *>(ws.q8) + ((long long)q.bh * ws.Nq_pad + q.r0) * Dp, Dp,
                   c8, rg, live, x, inv);
     }
