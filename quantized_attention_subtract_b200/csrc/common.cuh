@@ -134,22 +134,22 @@ __device__ __forceinline__ long long v_off(const Problem &pb, int b) {
   return pb.cu_kv ? (long long)pb.cu_kv[b] * pb.vs_n : (long long)b * pb.vs_b;
 }
 
-// Host-side launchers (defined in prepass.cu / attn_fwd.cu).
-// ---- INT8 codes (pre-pass and the attention kernel's fused Q path)
+// ---- integer codes of the pre-pass
 constexpr float kTinyAmax = 0x1p-64f;  // blocks below this quantise to zero
 
-// INT8 code of x with reciprocal scale inv: rint(fl(x * inv)), round half to
-// even.  Adding 1.5 * 2^23 in fp32 rounds to an integer exactly that way and
-// leaves it (two's complement) in the low mantissa bits; |fl(x * inv)| is at
-// most 127 * (1 + 2^-24), so the code is always in [-127, 127].
-__device__ __forceinline__ uint32_t int8_bits(float x, float inv) {
-  return __float_as_uint(__fadd_rn(__fmul_rn(x, inv), 12582912.0f));
-}
+// A code is rint(fl(x * inv)), round half to even: adding 1.5 * 2^23 in fp32
+// to fl(x * inv) rounds it to an integer exactly that way and leaves it (two's
+// complement) in the low mantissa bits; |fl(x * inv)| is at most
+// qmax * (1 + 2^-24), so the code stays in [-qmax, qmax].
+// The scalar __fmul_rn / __fadd_rn are never contracted into a fused
+// multiply-add; an f32x2 multiply followed by an f32x2 add can be (measured:
+// codes of exact ties moved), so codes are formed with scalar ops.
 // Pack the low bytes of four such words (first in bits [0, 8)).
 __device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
+// Host-side launchers (defined in prepass.cu / attn_fwd.cu).
 cudaError_t launch_prepass(const Problem &pb, const Workspace &ws, const InputMaps &im,
                            cudaStream_t stream);
 cudaError_t launch_attention(const Problem &pb, const Workspace &ws, const CUtensorMap &tm_q,

@@ -381,10 +381,11 @@ __device__ __forceinline__ void store_codes(uint8_t *dst, int Dp, int c8, int rg
   for (int r = 0; r < 4; ++r) {
     uint32_t w0 = 0u, w1 = 0u;
     if (live) {
-      w0 = pack4_lo(int8_bits(x[r][0], inv[r]), int8_bits(x[r][1], inv[r]),
-                    int8_bits(x[r][2], inv[r]), int8_bits(x[r][3], inv[r]));
-      w1 = pack4_lo(int8_bits(x[r][4], inv[r]), int8_bits(x[r][5], inv[r]),
-                    int8_bits(x[r][6], inv[r]), int8_bits(x[r][7], inv[r]));
+      uint32_t c[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c[e] = __float_as_uint(__fadd_rn(__fmul_rn(x[r][e], inv[r]), 12582912.0f));
+      w0 = pack4_lo(c[0], c[1], c[2], c[3]);
+      w1 = pack4_lo(c[4], c[5], c[6], c[7]);
     }
     if (8 * c8 < Dp) *reinterpret_cast<uint2 *>(dst + (4 * rg + r) * Dp + 8 * c8) = make_uint2(w0, w1);
   }
@@ -591,9 +592,11 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       for (int r = 0; r < 4; ++r)
         if (live && 4 * rg + r < q.nvalid)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x[r][e] = __fsub_rn(x[r][e], mean[e]);
-            a = fmaxf(a, fabsf(x[r][e]));
+          for (int e = 0; e < 8; e += 2) {
+            const float2 d = __fadd2_rn(make_float2(x[r][e], x[r][e + 1]), make_float2(-mean[e], -mean[e + 1]));
+            x[r][e] = d.x;
+            x[r][e + 1] = d.y;
+            a = fmaxf(a, fmaxf(fabsf(d.x), fabsf(d.y)));
           }
       // rows 32 k .. 32 k + 31 (row groups 8 k .. 8 k + 7) form block k; each
       // warp lies inside one block.  Non-negative floats order like their bits.
@@ -627,7 +630,12 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
       for (int r = 0; r < 4; ++r) {
         if (4 * rg + r < q.nvalid) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[r][e] = __fmul_rn(__fsub_rn(x[r][e], mean[e]), inv[e]);
+          for (int e = 0; e < 8; e += 2) {
+            const float2 d = __fmul2_rn(__fadd2_rn(make_float2(x[r][e], x[r][e + 1]), make_float2(-mean[e], -mean[e + 1])),
+                                     make_float2(inv[e], inv[e + 1]));
+            x[r][e] = d.x;
+            x[r][e + 1] = d.y;
+          }
         }
       }
       // Transposed tile [D][128 keys] as 32 words per channel row; the word of
@@ -689,7 +697,12 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
           for (int r = 0; r < 4; ++r)
             if (4 * rg + r < q.nvalid)
 #pragma unroll
-              for (int e = 0; e < 8; ++e) x[r][e] = __fsub_rn(x[r][e], chan[8 * c8 + e]);
+              for (int e = 0; e < 8; e += 2) {
+                const float2 d = __fadd2_rn(make_float2(x[r][e], x[r][e + 1]),
+                                         make_float2(-chan[8 * c8 + e], -chan[8 * c8 + e + 1]));
+                x[r][e] = d.x;
+                x[r][e + 1] = d.y;
+              }
         }
       }
       float a[4], inv[4];
