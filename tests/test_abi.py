@@ -247,3 +247,22 @@ def test_non_finite_sm_scale_rejected(scale):
     p = _params()
     p.sm_scale = scale
     assert _ws_size(p)[0] == 1
+
+
+def test_binding_passes_qk_bits():
+    """The Python builders fill sage_attn_params_t.qk_bits (default 8); the
+    library sizes the workspace the same for both code widths."""
+    import torch
+    q = torch.zeros(1, 2, 256, 64, dtype=torch.float16)
+    k = torch.zeros(1, 2, 256, 64, dtype=torch.float16)
+    p8 = binding.make_params(q, k, k, q)
+    p4 = binding.make_params(q, k, k, q, qk_bits=4)
+    assert p8.qk_bits == 8 and p4.qk_bits == 4
+    assert binding.workspace_bytes(p8) == binding.workspace_bytes(p4)
+    qv = torch.zeros(300, 2, 64, dtype=torch.bfloat16)
+    kv = torch.zeros(200, 2, 64, dtype=torch.bfloat16)
+    pv = binding.make_varlen_params(qv, kv, kv, qv, [0, 100, 300], [0, 50, 200], qk_bits=4)
+    assert pv.qk_bits == 4 and pv.B == 2
+    bad = binding.make_params(q, k, k, q, qk_bits=5)
+    with pytest.raises(binding.SageError):
+        binding.workspace_bytes(bad)
