@@ -6,8 +6,9 @@ library's static 64 MiB scratch instead of a caller workspace.
 Checked through the C ABI against sage_attn_fwd on the same inputs.  Both run
 the same kernels on the same inputs, so the outputs must be bit-identical.
 The calls come in a sequence that changes shape on the one shared array
-(large D = 128, then a ragged D = 96, then causal D = 64, then back), so stale
-padding, scales or accumulators left by a larger earlier call would show;
+(large D = 128, then a ragged D = 96, then causal D = 64, 4-bit Q/K codes,
+then back), so stale padding, scales or accumulators left by a larger earlier
+call would show;
 variable-length batches (sequence offsets and running totals in the scratch)
 and smoothed Q and V (the per-block means and the dS rows) are covered too.
 The device status the no-alloc path leaves is read back through its own
@@ -33,6 +34,7 @@ SEQUENCE = [
     ((1, 6, 3, 260, 261, 96), dict(dtype="fp16", layout="NHD")),
     ((1, 4, 1, 300, 300, 64), dict(dtype="bf16", is_causal=True)),
     ((1, 4, 2, 256, 640, 128), dict(dtype="fp16", smooth_q=True, smooth_v=True)),
+    ((1, 4, 2, 300, 500, 128), dict(dtype="bf16", qk_bits=4)),
     ((2, 4, 2, 900, 1400, 128), dict(dtype="bf16")),
 ]
 
@@ -41,7 +43,7 @@ def _pair(args, kw, seed):
     flags = {k: v for k, v in kw.items() if k in ("is_causal", "smooth_q", "smooth_v")}
     w = random_problem(*args, layout=kw.get("layout", "HND"), dtype=kw["dtype"], seed=seed, **flags)
     q, k, v = (to_device(x, w.dtype) for x in generate(w, seed))
-    fl = dict(smooth_q=w.smooth_q, smooth_v=w.smooth_v)
+    fl = dict(smooth_q=w.smooth_q, smooth_v=w.smooth_v, qk_bits=kw.get("qk_bits", 8))
     ref = torch.empty_like(q)
     p = binding.make_params(q, k, v, ref, w.layout, w.is_causal, None, True, **fl)
     ws = binding.alloc_workspace(p, q.device)
