@@ -55,3 +55,16 @@ def test_workload_full_size(name, smooth_k):
     else:
         bound = (EXACT_REL_L1, EXACT_COS)
     assert r["rel_l1_exact"] <= bound[0] and r["cos_exact"] >= bound[1], r
+
+
+def test_default_workload_full_size_int4():
+    """The benchmark's default workload with 4-bit Q/K codes (qk_bits = 4):
+    pre-pass bit for bit, output against the 4-bit oracle at the same bounds,
+    and no worse against exact attention than the 4-bit method itself."""
+    w = WORKLOADS["gqa_causal_n32768_d128_bf16"].with_(qk_bits=4)
+    q, k, v, pr, pre, g = run_both(w)
+    assert_prepass_bit_exact(w, pre, g)
+    r = compare_output(pr, pre, q, k, v, g, sample_tiles(pr, 6, seed=2))
+    assert r["max_abs_excess"] <= MIRROR_MAX_ABS and r["cos"] >= MIRROR_COS, r
+    assert r["rel_l1_exact"] <= r["mirror_rel_l1_exact"] + 0.002, r
+    assert r["cos_exact"] >= r["mirror_cos_exact"] - 0.0005, r
