@@ -144,7 +144,8 @@ constexpr float kTinyAmax = 0x1p-64f;  // blocks below this quantise to zero
 // The scalar __fmul_rn / __fadd_rn are never contracted into a fused
 // multiply-add; an f32x2 multiply followed by an f32x2 add can be (measured:
 // codes of exact ties moved), so codes are formed with scalar ops.
-// Pack the low bytes of four such words (first in bits [0, 8)).
+
+// Pack the low bytes of four such code words (first in bits [0, 8)).
 __device__ __forceinline__ uint32_t pack4_lo(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }

@@ -699,7 +699,7 @@ __global__ void __launch_bounds__(512, 2) quantize_kernel(Problem pb, Workspace 
 #pragma unroll
               for (int e = 0; e < 8; e += 2) {
                 const float2 d = __fadd2_rn(make_float2(x[r][e], x[r][e + 1]),
-                                         make_float2(-chan[8 * c8 + e], -chan[8 * c8 + e + 1]));
+                                            make_float2(-chan[8 * c8 + e], -chan[8 * c8 + e + 1]));
                 x[r][e] = d.x;
                 x[r][e + 1] = d.y;
               }
