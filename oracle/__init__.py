@@ -290,8 +290,8 @@ def varlen_attention(Hq: int, Hkv: int, D: int, cu_q, cu_kv, q: np.ndarray, k: n
                      smooth_k: bool = True, smooth_q: bool = False, smooth_v: bool = False,
                      sm_scale: float | None = None, with_uncertainty: bool = False,
                      exact: bool = False, qk_bits: int = 8) -> dict:
-    """A variable-length batch of packed sequences ("variable sequence lengths
-    per batch", sageattention package page): sequence b is rows
+    """A variable-length batch of packed sequences (the sageattention package
+    page lists batches whose sequences differ in length): sequence b is rows
     cu_q[b] .. cu_q[b+1] of q [total_q, Hq, D] attending to rows
     cu_kv[b] .. cu_kv[b+1] of k, v [total_kv, Hkv, D], and nothing else.
     The pages fix no more than that; the reading taken is that each sequence
